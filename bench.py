@@ -1,0 +1,360 @@
+"""Benchmark of the per-step top-k sparse-attention decode path on B200.
+
+Default workload (one GPU): the Qwen3-8B-shaped 128K decode layer -- 16
+requests, 8 KV heads of 4 query heads, d = 128, 131072 keys each, a 92-bit
+Fathom budget per key, top-2048 per (request, KV head), a 4096-entry hot
+buffer per (request, KV head) holding 80% of the selection. One step is one
+fused decode_step over the whole batch: bit allocation, bit-plane scan, top-k,
+slot lookup and sparse GQA attention.
+
+metric: keys scored per second by the full decode step (each step scores
+R*G*n keys); layer-steps/s and achieved HBM GB/s are reported beside it.
+Inputs are synthetic (seeded draws with the pages' shapes and distributions)
+and stay resident in HBM; every step reads ~350 MB, more than the 126 MB L2,
+so no L2 flush is needed between steps.
+
+--impl reference times the CPU oracle (the only reference this method has) on
+a bounded sample of the same workload, on the host cores.
+Multi-GPU (torchrun): independent replicas, one per GPU (weak scaling); no
+collective is on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOADS = {
+    # name: R, G, H, n, B, k, S, miss fraction
+    "qwen3-8b-128k": dict(R=16, G=8, H=4, n=131072, B=92, k=2048, S=4096, miss=0.2),
+    "qwen3-8b-1m": dict(R=4, G=8, H=4, n=1048576, B=92, k=2048, S=4096, miss=0.2),
+    "tiny": dict(R=1, G=1, H=4, n=4096, B=92, k=256, S=512, miss=0.2),
+}
+METRIC = "index-scan keys/s + sparse decode layer-steps/s; achieved GB/s vs HBM peak"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1:
+        import torch.distributed as dist
+        import datetime
+        rank = int(os.environ["RANK"])
+        local = int(os.environ.get("LOCAL_RANK", rank))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist, rank, ws
+    return None, 0, 1
+
+
+def _max_over_ranks(dist, x: float) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    def __init__(self):
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        dev = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0] or str(torch.cuda.current_device())
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={dev}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def setup(cfg: dict, device, seed: int = 1):
+    """Synthetic inputs resident on the device, a warm-up selection, and the hot
+    buffers built around it (80% of the selected rows present)."""
+    import kv_index_scan_b200 as kvs
+    R, G, H, n, B, k, S = (cfg[x] for x in ("R", "G", "H", "n", "B", "k", "S"))
+    K, V, nl = synth.fathom_kv(R, G, 128, n, seed=seed, device=device)
+    q = synth.queries(R, G, H, 128, seed=seed, device=device)
+    index = kvs.build_fathom_index(K, nl)
+    warm = kvs.DecodeStep(index, nl, n, H, B, k, K, V)
+    warm(q)
+    torch.cuda.synchronize()
+    sel = warm.idx.cpu().numpy()
+    del warm
+    slot_map, hot_tok = synth.slot_map_from_selection(sel, nl, n, S, cfg["miss"], seed=seed)
+    hotK, hotV = synth.hot_rows(K, hot_tok), synth.hot_rows(V, hot_tok)
+    slot_map_t = torch.from_numpy(slot_map).to(device)
+    step = kvs.DecodeStep(index, nl, n, H, B, k, K, V, slot_map_t, hotK, hotV)
+    return dict(K=K, V=V, q=q, index=index, step=step, nl=nl, slot_map=slot_map_t, hotK=hotK,
+                hotV=hotV, sel=sel)
+
+
+def algorithmic_bytes(cfg: dict) -> dict:
+    R, G, n, B, k = (cfg[x] for x in ("R", "G", "n", "B", "k"))
+    keys = R * G * n
+    scan = keys * B / 8
+    rows = R * G * k * (2 * 128 * 2 + 32)  # K + V rows and one 32-byte slot-map sector
+    return dict(keys=keys, scan=scan, rows=rows, total=scan + rows)
+
+
+def time_steps(fn, steps: int, warmup: int, stream) -> float:
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def run_ours(args, cfg, dist, rank, ws):
+    import kv_index_scan_b200 as kvs
+    dev = torch.device("cuda", torch.cuda.current_device())
+    data = setup(cfg, dev, seed=1 + rank)
+    step, q = data["step"], data["q"]
+    stream = torch.cuda.current_stream()
+    algo = algorithmic_bytes(cfg)
+
+    # ---- device-resident timed region: whole decode steps ----
+    for _ in range(args.warmup):
+        step(q)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = Clocks()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(q)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    clk = clocks.stop()
+    if dist:
+        dist.barrier()
+    ms_max = _max_over_ranks(dist, ms)
+
+    # ---- dominant kernel alone (the bit-plane scan), same stream, CUDA events ----
+    scan_scores = torch.empty(cfg["R"], cfg["G"], cfg["n"], dtype=torch.float32, device=dev)
+    plan = step.plan
+
+    def scan_once():
+        kvs.index_scan_fathom(data["index"], plan, data["nl"], cfg["n"], scores=scan_scores)
+
+    scan_ms = time_steps(scan_once, max(args.steps, 5), 3, stream)
+
+    # ---- end to end through the C ABI with host buffers ----
+    R, G, H = cfg["R"], cfg["G"], cfg["H"]
+    q_host = q.cpu().pin_memory()
+    out_host = torch.empty(R, G, H, 128, dtype=torch.float32).pin_memory()
+    idx_host = torch.empty(R, G, cfg["k"], dtype=torch.int32).pin_memory()
+    miss_host = torch.empty(R, G, dtype=torch.int32).pin_memory()
+    q_dev = torch.empty_like(q)
+
+    def e2e_once():
+        q_dev.copy_(q_host, non_blocking=True)
+        step(q_dev)
+        out_host.copy_(step.out, non_blocking=True)
+        idx_host.copy_(step.idx, non_blocking=True)
+        miss_host.copy_(step.misses, non_blocking=True)
+
+    e2e_ms = _max_over_ranks(dist, time_steps(e2e_once, args.steps, args.warmup, stream))
+    h2d = q_host.numel() * 4
+    d2h = out_host.numel() * 4 + idx_host.numel() * 4 + miss_host.numel() * 4
+    misses = int(step.misses.sum().item())
+
+    peak, peak_kind = _peaks()
+    keys_total = algo["keys"] * ws
+    value = keys_total / (ms_max / 1e3)
+    scan_bytes = algo["scan"]
+    scan_gbs = scan_bytes / (scan_ms / 1e3) / 1e9
+    launches_per_step = 5 + (1 if step_needs_combine(cfg) else 0)
+    res = {
+        "metric": METRIC, "value": value, "unit": "keys/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": args.workload, "requests": R, "kv_heads": G, "q_heads_per_kv": H,
+                   "head_dim": 128, "context": cfg["n"], "bits_per_key": cfg["B"],
+                   "topk": cfg["k"], "hot_slots": cfg["S"], "miss_rate": cfg["miss"],
+                   "parallelism": f"replicas{ws}" if ws > 1 else "single",
+                   "l2": "inputs larger than L2 (>=350 MB read per step)"},
+        "layer_steps_per_s": ws * 1e3 / ms_max,
+        "achieved_gbs": algo["total"] * ws / (ms_max / 1e3) / 1e9,
+        "miss_rate_measured": misses / (R * G * cfg["k"]),
+        "roofline": {"bound": "hbm", "kernel": "fathom_scan", "achieved": scan_gbs, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": scan_gbs / peak,
+                     "traffic": None, "algorithmic_bytes": scan_bytes, "ms": scan_ms},
+        "e2e": {"value": keys_total / (e2e_ms / 1e3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(cfg, data, rows=args.cpu_rows)
+    return res
+
+
+def step_needs_combine(cfg) -> bool:
+    import kv_index_scan_b200 as kvs
+    return kvs._lib.kvs_attn_workspace_size(cfg["R"], cfg["G"], cfg["H"], cfg["k"]) > 0
+
+
+def cpu_baseline(cfg, data, rows: int = 8) -> dict:
+    """The CPU oracle, as it stands, on a bounded sample of the same workload:
+    `rows` (request, KV head) rows of the decode step, all host cores."""
+    import oracle
+    R, G, H, n, B, k = (cfg[x] for x in ("R", "G", "H", "n", "B", "k"))
+    rows = min(rows, R * G)
+    us = list(range(rows))
+    rr = [u // G for u in us]
+    gg = [u % G for u in us]
+    K = data["K"][rr, gg].unsqueeze(0).cpu()
+    V = data["V"][rr, gg].unsqueeze(0).cpu()
+    q = data["q"][rr, gg].unsqueeze(0).cpu()
+    nl = [data["nl"][0]]
+    sm = data["slot_map"][rr, gg].unsqueeze(0).cpu()
+    hK = data["hotK"][rr, gg].unsqueeze(0).cpu()
+    hV = data["hotV"][rr, gg].unsqueeze(0).cpu()
+    W = synth.plane_words(n)
+    planes, kmin, kstep, kvar = oracle.build_index_batch(K, nl, W)  # data prep, not timed
+    cores = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    oracle.decode_batch(q, planes, kmin, kstep, kvar, nl, B, k, sm, hK, hV, K, V,
+                        1 / math.sqrt(128), nthreads=cores)
+    dt = time.perf_counter() - t0
+    return {"value": rows * n / dt, "unit": "keys/s", "cores": cores, "kind": "oracle",
+            "sample": f"{rows} of {R * G} (request, KV head) rows of one decode step "
+                      f"({rows * n} keys), fp64 C++ oracle, {dt:.2f} s"}
+
+
+def run_reference(args, cfg, dist, rank, ws):
+    """The CPU oracle timed as the reference arm, on the same workload's shape."""
+    import oracle
+    dev = torch.device("cuda", torch.cuda.current_device()) if torch.cuda.is_available() else "cpu"
+    R, G, H, n, B, k, S = (cfg[x] for x in ("R", "G", "H", "n", "B", "k", "S"))
+    rows = min(args.cpu_rows, R * G)
+    # a sample of rows of the same workload: (rows requests x 1 head) of length n
+    K, V, nl = synth.fathom_kv(rows, 1, 128, n, seed=1)
+    q = synth.queries(rows, 1, H, 128, seed=1)
+    W = synth.plane_words(n)
+    planes, kmin, kstep, kvar = oracle.build_index_batch(K, nl, W)
+    cores = os.cpu_count() or 1
+    ref0 = oracle.decode_batch(q, planes, kmin, kstep, kvar, nl, B, k, None, None, None, K, V,
+                               1 / math.sqrt(128), nthreads=cores)
+    slot_map, hot_tok = synth.slot_map_from_selection(ref0["idx"], nl, n, S, cfg["miss"], seed=1)
+    hK, hV = synth.hot_rows(K, hot_tok), synth.hot_rows(V, hot_tok)
+
+    def one():
+        oracle.decode_batch(q, planes, kmin, kstep, kvar, nl, B, k, slot_map, hK, hV, K, V,
+                            1 / math.sqrt(128), nthreads=cores)
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    dt = (time.perf_counter() - t0) / args.steps
+    v = rows * n / dt
+    return {"metric": METRIC, "value": v, "unit": "keys/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": args.workload, "requests": R, "kv_heads": G,
+                       "q_heads_per_kv": H, "head_dim": 128, "context": n, "bits_per_key": B,
+                       "topk": k, "hot_slots": S, "miss_rate": cfg["miss"]},
+            "cpu_baseline": {"value": v, "unit": "keys/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{rows} (request, KV head) rows of {n} keys per step"},
+            "e2e": {"value": v, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="qwen3-8b-128k", choices=sorted(WORKLOADS))
+    ap.add_argument("--B", type=int, default=None, help="bits per key (default: the workload's)")
+    ap.add_argument("--cpu-rows", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = dict(WORKLOADS[args.workload])
+    if args.B is not None:
+        cfg["B"] = args.B
+    if args.impl == "reference":
+        # the CPU oracle: rank 0 alone runs it; other ranks exit without work
+        if int(os.environ.get("RANK", "0")) == 0:
+            ws = int(os.environ.get("WORLD_SIZE", "1"))
+            print(json.dumps(run_reference(args, cfg, None, 0, ws)), flush=True)
+        return
+    dist, rank, ws = _dist()
+    res = run_ours(args, cfg, dist, rank, ws)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -67,6 +67,12 @@ extern "C" {
 
 #define KVS_ABI_VERSION 1
 
+#if defined(__GNUC__)
+#define KVS_API __attribute__((visibility("default")))
+#else
+#define KVS_API
+#endif
+
 typedef int32_t kvs_status;
 enum {
   KVS_OK = 0,
@@ -82,9 +88,9 @@ enum { KVS_F32 = 0, KVS_BF16 = 1 };              /* q dtypes              */
 enum { KVS_SCAN_FATHOM = 0, KVS_SCAN_LIGHTNING = 1 };
 
 /* Returns KVS_ABI_VERSION of the loaded library. */
-int32_t kvs_abi_version(void);
+KVS_API int32_t kvs_abi_version(void);
 /* Thread-local text of the last error returned on this thread ("" if none). */
-const char* kvs_last_error(void);
+KVS_API const char* kvs_last_error(void);
 
 /* ---------------------------------------------------------------------------
  * The Fathom K index [FATHOM].
@@ -123,11 +129,11 @@ typedef struct {
 /* a0: quantise K (bf16 [R][G][n_max][D], token-major) into the index above.
  * D must be 128. Codes are decided in fp64 exactly as written above, so the
  * result is bit-reproducible. Workspace: kvs_build_index_workspace_size(). */
-kvs_status kvs_build_fathom_index(const uint16_t* K, const int32_t* n, int32_t R, int32_t G,
+KVS_API kvs_status kvs_build_fathom_index(const uint16_t* K, const int32_t* n, int32_t R, int32_t G,
                                   int32_t n_max, int32_t D, int32_t W, uint32_t* planes,
                                   float* kmin, float* kstep, float* kvar, void* ws,
                                   size_t ws_bytes, int32_t* dev_status, void* stream);
-size_t kvs_build_index_workspace_size(int32_t R, int32_t G, int32_t D);
+KVS_API size_t kvs_build_index_workspace_size(int32_t R, int32_t G, int32_t D);
 
 /* ---------------------------------------------------------------------------
  * a1: per-query bit allocation [FATHOM]: reverse water-filling of the bit
@@ -158,7 +164,7 @@ typedef struct {
   int32_t B;
 } kvs_plan;
 
-kvs_status fathom_plan_bits(const float* q /* f32 [R][G][H][D] */, int32_t H,
+KVS_API kvs_status fathom_plan_bits(const float* q /* f32 [R][G][H][D] */, int32_t H,
                             const kvs_fathom_index* ix, int32_t B, const kvs_plan* plan,
                             int32_t* dev_status, void* stream);
 
@@ -194,7 +200,7 @@ typedef struct {
   int32_t Hi, Dl, block;
 } kvs_scan_args;
 
-kvs_status index_scan(const kvs_scan_args* a, float* scores, int32_t* dev_status, void* stream);
+KVS_API kvs_status index_scan(const kvs_scan_args* a, float* scores, int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------
  * a3: exact top-k [XMSPARSE: 2,048 entries chosen per layer and step;
@@ -210,10 +216,10 @@ kvs_status index_scan(const kvs_scan_args* a, float* scores, int32_t* dev_status
  * vals (nullable) f32 [R][G][k]: the score of each output (token score, or
  *   the block's score in block mode), -inf for padding.
  * NaN scores are not supported. Workspace: kvs_topk_workspace_size(). */
-kvs_status topk_select(const float* scores, int64_t ld, const int32_t* n, int32_t R, int32_t G,
+KVS_API kvs_status topk_select(const float* scores, int64_t ld, const int32_t* n, int32_t R, int32_t G,
                        int32_t k, int32_t block, int32_t* idx, float* vals, void* ws,
                        size_t ws_bytes, int32_t* dev_status, void* stream);
-size_t kvs_topk_workspace_size(int32_t R, int32_t G, int32_t n_max, int32_t k, int32_t block);
+KVS_API size_t kvs_topk_workspace_size(int32_t R, int32_t G, int32_t n_max, int32_t k, int32_t block);
 
 /* ---------------------------------------------------------------------------
  * a4: gather the selected K/V rows [XMSPARSE, Figure 1 and the lifecycle
@@ -229,7 +235,7 @@ size_t kvs_topk_workspace_size(int32_t R, int32_t G, int32_t n_max, int32_t k, i
  *   idx i32 [R][G][k]; slot_map i32 [R][G][n_max]; hot bf16 [R][G][S][D];
  *   full bf16 [R][G][n_max][D]; gK/gV bf16 [R][G][k][D]; slots i32 [R][G][k];
  *   misses i32 [R][G]. D = 128. */
-kvs_status sparse_gather(const int32_t* idx, int32_t k, const int32_t* slot_map,
+KVS_API kvs_status sparse_gather(const int32_t* idx, int32_t k, const int32_t* slot_map,
                          const uint16_t* hotK, const uint16_t* hotV, int32_t S,
                          const uint16_t* fullK, const uint16_t* fullV, const int32_t* n,
                          int32_t n_max, int32_t R, int32_t G, int32_t D, uint16_t* gK,
@@ -245,12 +251,12 @@ kvs_status sparse_gather(const int32_t* idx, int32_t k, const int32_t* slot_map,
  * out f32 [R][G][H][D]; lse (nullable) f32 [R][G][H] = log sum_j exp(l_j)
  * (natural log). A head with k_eff = 0 gets out = 0 and lse = -inf.
  * D = 128, H in 1..8. Workspace: kvs_attn_workspace_size(). */
-kvs_status sparse_decode_attn(const void* q, int32_t q_dtype, const uint16_t* K,
+KVS_API kvs_status sparse_decode_attn(const void* q, int32_t q_dtype, const uint16_t* K,
                               const uint16_t* V, const int32_t* k_eff, int32_t R, int32_t G,
                               int32_t H, int32_t D, int32_t k, float scale, float* out,
                               float* lse, void* ws, size_t ws_bytes, int32_t* dev_status,
                               void* stream);
-size_t kvs_attn_workspace_size(int32_t R, int32_t G, int32_t H, int32_t k);
+KVS_API size_t kvs_attn_workspace_size(int32_t R, int32_t G, int32_t H, int32_t k);
 
 /* ---------------------------------------------------------------------------
  * a6: one fused decode step for all (r, g), on one stream.
@@ -292,9 +298,9 @@ typedef struct {
   int32_t* misses;
 } kvs_decode_args;
 
-kvs_status decode_step(const kvs_decode_args* a, void* ws, size_t ws_bytes, int32_t* dev_status,
+KVS_API kvs_status decode_step(const kvs_decode_args* a, void* ws, size_t ws_bytes, int32_t* dev_status,
                        void* stream);
-size_t kvs_decode_step_workspace_size(int32_t R, int32_t G, int32_t H, int32_t n_max, int32_t k,
+KVS_API size_t kvs_decode_step_workspace_size(int32_t R, int32_t G, int32_t H, int32_t n_max, int32_t k,
                                       int32_t B);
 
 #ifdef __cplusplus

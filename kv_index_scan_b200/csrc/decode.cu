@@ -1,0 +1,100 @@
+// decode.cu -- a6: one fused decode step for every (request, KV head), and
+// the dispatch of the index scans.
+//
+// Step order (all on the caller's stream, nothing synchronised):
+//   plan_bits -> Fathom scan -> top-k -> slots + misses -> attention over
+//   the selected rows read through the slot map.
+// With a selection given (idx_in), the first three are skipped: the layer
+// group sharing of "MiniMax-M3: share the sparse index top-k across layers and
+// reuse the decode top-k buffer" (description), where the group's first layer
+// selects and the others reuse the selection.
+#include "internal.cuh"
+#include "scan_core.cuh"
+
+namespace kvs {
+
+kvs_status fathom_scan_dispatch(const kvs_fathom_index* ix, const kvs_plan* plan,
+                                const int32_t* n, int n_max, float* scores, int32_t* dev_status,
+                                cudaStream_t s) {
+  if (ix->host_mapped || plan->B == 0)
+    return fathom_scan_simple_launch(ix->planes, ix->W, ix->R, ix->G, plan->plane_idx,
+                                     plan->plane_w, plan->C, plan->B, n, n_max, scores, s);
+  ScanParams p{};
+  p.planes = ix->planes;
+  p.W = ix->W;
+  p.RG = ix->R * ix->G;
+  p.Gheads = ix->G;
+  p.plane_idx = plan->plane_idx;
+  p.plane_w = plan->plane_w;
+  p.C = plan->C;
+  p.B = plan->B;
+  p.n = n;
+  p.n_max = n_max;
+  scan_schedule(plan->B, p.G, p.b, p.nsets);
+  p.chunks_per_row = ((n_max + 31) / 32 + kChunkWords - 1) / kChunkWords;
+  p.scores = scores;
+  p.dev_status = dev_status;
+  return fathom_scan_lut_launch(p, s);
+}
+
+size_t decode_ws_bytes(int R, int G, int H, int n_max, int k, int B) {
+  (void)B;
+  WsCarver c(nullptr);
+  c.take<float>(static_cast<size_t>(R) * G * n_max);  // scores
+  c.take<int32_t>(static_cast<size_t>(R) * G * k);    // slots when the caller passes none
+  c.take<unsigned char>(attn_ws_bytes(R * G, H, k));
+  return c.used;
+}
+
+kvs_status decode_step_run(const kvs_decode_args* a, void* ws, int32_t* dev_status,
+                           cudaStream_t s) {
+  const int R = a->ix->R, G = a->ix->G, RG = R * G;
+  WsCarver c(ws);
+  float* scores = c.take<float>(static_cast<size_t>(RG) * a->n_max);
+  int32_t* slots_ws = c.take<int32_t>(static_cast<size_t>(RG) * a->k);
+  void* attn_ws = c.take<unsigned char>(attn_ws_bytes(RG, a->H, a->k));
+  kvs_status st;
+  const int32_t* sel = a->idx_in;
+  int shared = a->idx_in ? a->idx_shared : 0;
+  if (!sel) {
+    st = plan_bits_launch(static_cast<const float*>(a->q), a->H, a->ix->kmin, a->ix->kstep,
+                          a->ix->kvar, RG, a->plan->B, a->plan->t, a->plan->plane_idx,
+                          a->plan->plane_w, a->plan->C, s);
+    if (st != KVS_OK) return st;
+    st = fathom_scan_dispatch(a->ix, a->plan, a->n, a->n_max, scores, dev_status, s);
+    if (st != KVS_OK) return st;
+    st = topk_launch(scores, a->n_max, a->n, R, G, a->k, 1, a->idx, nullptr, s);
+    if (st != KVS_OK) return st;
+    sel = a->idx;
+  }
+  int32_t* slots = a->slots ? a->slots : slots_ws;
+  st = select_slots_launch(sel, shared, G, a->k, a->slot_map, a->n_max, RG, slots, a->misses, s);
+  if (st != KVS_OK) return st;
+  RowSrc src{};
+  src.mode = a->slot_map ? kRowsSlot : kRowsDirect;
+  src.K = a->fullK;
+  src.V = a->fullV;
+  src.hotK = a->hotK;
+  src.hotV = a->hotV;
+  src.idx = sel;
+  src.idx_shared = shared;
+  src.slots = slots;
+  src.slot_map = a->slot_map;
+  src.n_max = a->n_max;
+  src.S = a->S;
+  src.G = G;
+  src.k = a->k;
+  return attn_launch(a->q, a->q_dtype == KVS_BF16, src, RG, a->H, a->scale, a->out, a->lse,
+                     attn_ws, s);
+}
+
+kvs_status lightning_scan_dispatch(const kvs_scan_args* a, float* scores, int32_t* dev_status,
+                                   cudaStream_t s) {
+  (void)a;
+  (void)scores;
+  (void)dev_status;
+  (void)s;
+  return fail(KVS_EUNSUPPORTED, "index_scan: the lightning indexer is not built yet");
+}
+
+}  // namespace kvs

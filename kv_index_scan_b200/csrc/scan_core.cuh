@@ -1,0 +1,354 @@
+// scan_core.cuh -- the warp-specialised core of the HBM Fathom scan (see
+// scan_lut.cu for the method): TMA bulk staging of plane segments, in-register
+// 32x32 bit transposes, and bank-rotated group lookup tables. The epilogue
+// (write scores, or keep top-k candidates) is supplied by the kernel.
+#pragma once
+
+#include "internal.cuh"
+
+namespace kvs {
+
+constexpr int kScanConsumerWarps = 4;
+constexpr int kScanThreads = 32 * (kScanConsumerWarps + 1);  // + one producer warp
+constexpr int kChunkWords = 32 * kScanConsumerWarps;          // one 32-key word per consumer thread
+constexpr int kRowBytes = 4 * kChunkWords;                    // 512 bytes of a plane per chunk
+constexpr long long kWaitCycles = 2000000000ll;               // ~1 s bound on every wait
+
+struct ScanParams {
+  const uint32_t* planes;  // [RG][D][4][W]
+  int W;
+  int RG, Gheads;  // rows (r, g), and KV heads per request (row u belongs to request u / Gheads)
+  const uint16_t* plane_idx;  // [RG][B]
+  const float* plane_w;       // [RG][B]
+  const float* C;             // [RG]
+  int B;
+  const int32_t* n;
+  int n_max;
+  int G, b, nsets;  // lookup schedule: G groups of b planes per set
+  int chunks_per_row;
+  float* scores;  // unfused output [RG][n_max]
+  int32_t* dev_status;
+  // fused top-k candidates (scan_topk.cu)
+  int k;
+  int segs_per_row;
+  uint32_t* cand_key;   // [RG][segs][k]
+  int32_t* cand_idx;    // [RG][segs][k]
+  int32_t* cand_count;  // [RG][segs]
+};
+
+// Picks the lookup schedule for a budget of B planes: the fewest groups per
+// set with tables of at most 2^9 entries.
+inline void scan_schedule(int B, int& G, int& b, int& nsets) {
+  if (B <= 72) {
+    G = 8;
+    b = B <= 0 ? 1 : (B + 7) / 8;
+    nsets = 1;
+  } else if (B <= 144) {
+    G = 16;
+    b = (B + 15) / 16;
+    nsets = 1;
+  } else {
+    G = 16;
+    b = 6;
+    nsets = (B + 95) / 96;
+  }
+}
+
+// A zero plane segment in global memory: the source of padding slots.
+__device__ __align__(16) uint32_t kZeroRow[kChunkWords];
+
+// Dynamic shared memory of the scan kernels: [tables | stages | barriers].
+// Indexing this symbol directly keeps every table lookup a shared-memory load
+// with the base folded into the address.
+extern __shared__ __align__(1024) unsigned char g_scan_smem[];
+
+// ----------------------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait on a phase: false when about one second passes without it.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) return false;
+  }
+  return true;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, %0;\n" ::"n"(32 * kScanConsumerWarps) : "memory");
+}
+
+// 32x32 bit transpose in registers: afterwards bit c of x[r] is bit r of the
+// original x[c]. Byte-level stages with byte permutes, bit-level stages with
+// a shift and a bit select each.
+__device__ __forceinline__ void transpose32(uint32_t (&x)[32]) {
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const uint32_t a = x[k], c = x[k + 16];
+    x[k] = __byte_perm(a, c, 0x5410);
+    x[k + 16] = __byte_perm(a, c, 0x7632);
+  }
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    if (k & 8) continue;
+    const uint32_t a = x[k], c = x[k + 8];
+    x[k] = __byte_perm(a, c, 0x6240);
+    x[k + 8] = __byte_perm(a, c, 0x7351);
+  }
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    if (k & 4) continue;
+    const uint32_t t = ((x[k] >> 4) ^ x[k + 4]) & 0x0F0F0F0Fu;
+    x[k + 4] ^= t;
+    x[k] ^= t << 4;
+  }
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    if (k & 2) continue;
+    const uint32_t t = ((x[k] >> 2) ^ x[k + 2]) & 0x33333333u;
+    x[k + 2] ^= t;
+    x[k] ^= t << 2;
+  }
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    if (k & 1) continue;
+    const uint32_t t = ((x[k] >> 1) ^ x[k + 1]) & 0x55555555u;
+    x[k + 1] ^= t;
+    x[k] ^= t << 1;
+  }
+}
+
+template <int G, int b>
+struct ScanCore {
+  static constexpr int NPOS = G * b;            // plane slots per set
+  static constexpr int NBLK = (NPOS + 31) / 32;  // 32-plane transposes per set
+  static constexpr int TBL_BYTES = (1 << b) * 128;
+  static constexpr int STAGE_BYTES = NPOS * kRowBytes;
+
+  __host__ __device__ static int nstages(int nsets) {
+    const int budget = 220 * 1024 - nsets * TBL_BYTES - 256;
+    int s = budget / STAGE_BYTES;
+    return s > 4 ? 4 : s;
+  }
+  __host__ __device__ static size_t smem_bytes(int nsets) {
+    return static_cast<size_t>(nsets) * TBL_BYTES + static_cast<size_t>(nstages(nsets)) * STAGE_BYTES +
+           256;
+  }
+
+  const ScanParams& p;
+  int nstage;
+  unsigned char* stages;
+  uint64_t* full;
+  uint64_t* empty;
+  int* abort_flag;
+
+  __device__ explicit ScanCore(const ScanParams& params) : p(params) {
+    nstage = nstages(p.nsets);
+    stages = g_scan_smem + p.nsets * TBL_BYTES;
+    full = reinterpret_cast<uint64_t*>(stages + nstage * STAGE_BYTES);
+    empty = full + nstage;
+    abort_flag = reinterpret_cast<int*>(empty + nstage);
+  }
+
+  __device__ void fail_timeout() {
+    set_status(p.dev_status, KVS_ETIMEOUT);
+    atomicExch(abort_flag, 1);
+  }
+
+  // item -> (row u, chunk c, set s)
+  __device__ void decode_item(int it, int& u, int& c, int& s) const {
+    s = it % p.nsets;
+    const int rc = it / p.nsets;
+    c = rc % p.chunks_per_row;
+    u = rc / p.chunks_per_row;
+  }
+
+  __device__ void produce(int beg, int end) {
+    const int lane = threadIdx.x & 31;
+    int issued = 0;
+    for (int it = beg; it < end; ++it) {
+      const int k = it - beg, st = k % nstage;
+      if (k >= nstage && !mbar_wait(&empty[st], ((k / nstage) - 1) & 1)) {
+        if (lane == 0) fail_timeout();
+        break;
+      }
+      if (*reinterpret_cast<volatile int*>(abort_flag)) break;
+      int u, c, s;
+      decode_item(it, u, c, s);
+      const int w0 = c * kChunkWords;
+      const int nr = p.n[u / p.Gheads];
+      const bool live = 32 * w0 < nr;
+      const int words = min(kChunkWords, p.W - w0);
+      const uint32_t bytes = live ? static_cast<uint32_t>(words) * 4u : 0u;
+      if (lane == 0) mbar_expect_tx(&full[st], bytes * NPOS);
+      __syncwarp();
+      if (live) {
+        unsigned char* dst0 = stages + st * STAGE_BYTES;
+        const uint32_t* rowp = p.planes + static_cast<size_t>(u) * kD * 4 * p.W + w0;
+        const uint16_t* pidx = p.plane_idx + static_cast<size_t>(u) * p.B;
+        for (int q = lane; q < NPOS; q += 32) {
+          const int slot = s * NPOS + q;
+          const uint32_t* src =
+              slot < p.B ? rowp + static_cast<size_t>(pidx[slot]) * p.W : kZeroRow;
+          bulk_g2s(dst0 + q * kRowBytes, src, bytes, &full[st]);
+        }
+      }
+      ++issued;
+    }
+    // drain: never leave copies in flight into this block's shared memory
+    for (int k = max(0, issued - nstage); k < issued; ++k)
+      mbar_wait(&full[k % nstage], (k / nstage) & 1);
+  }
+
+  __device__ void build_tables(int u) {
+    const int t = threadIdx.x;
+    const float* w = p.plane_w + static_cast<size_t>(u) * p.B;
+    const int entries = p.nsets * (1 << b) * 32;
+    for (int e = t; e < entries; e += 32 * kScanConsumerWarps) {
+      const int slot = e & 31;
+      const int idx = (e >> 5) & ((1 << b) - 1);
+      const int s = e >> (5 + b);
+      const int base = s * NPOS + (slot % G) * b;
+      float v = 0.f;
+#pragma unroll
+      for (int bi = 0; bi < b; ++bi)
+        if (((idx >> bi) & 1) && base + bi < p.B) v += w[base + bi];
+      *reinterpret_cast<float*>(g_scan_smem + s * TBL_BYTES + idx * 128 + slot * 4) = v;
+    }
+  }
+
+  // The set's contribution for this thread's 32 keys, added into acc.
+  __device__ __forceinline__ void compute_set(int stage_off, int s, float (&acc)[32]) const {
+    const int t = threadIdx.x;
+    const int lane = t & 31;
+    const int lp = lane % G, repl = lane / G;
+    const unsigned char* mine = g_scan_smem + stage_off + 4 * t;
+    uint32_t prev[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) prev[j] = 0u;
+#pragma unroll
+    for (int m = 0; m < NBLK; ++m) {
+      uint32_t x[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        const int o = 32 * m + q;
+        if (o < NPOS) {
+          const int g = o / b, bi = o % b;
+          const int gr = (g + lp) & (G - 1);
+          x[q] = *reinterpret_cast<const uint32_t*>(mine + (gr * b + bi) * kRowBytes);
+        } else {
+          x[q] = 0u;
+        }
+      }
+      transpose32(x);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const int st = g * b, en = st + b - 1;
+        if ((en >> 5) != m) continue;
+        const int sh = st & 31;
+        const bool straddle = (st >> 5) != m;
+        const uint32_t rs = static_cast<uint32_t>((((g + lp) & (G - 1)) + G * repl) * 4 +
+                                                  s * TBL_BYTES);
+        constexpr uint32_t mask7 = ((1u << b) - 1u) << 7;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          uint32_t v;
+          if (straddle)
+            v = __funnelshift_r(prev[j], x[j], sh - 7);
+          else if (sh >= 7)
+            v = x[j] >> (sh - 7);
+          else
+            v = x[j] << (7 - sh);
+          const uint32_t addr = (v & mask7) | rs;
+          acc[j] += *reinterpret_cast<const float*>(g_scan_smem + addr);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) prev[j] = x[j];
+    }
+  }
+
+  // Runs the pipeline over this block's items; epi(u, w0, nr, acc, t) is
+  // called by every consumer thread at the end of each chunk.
+  template <typename Epi>
+  __device__ void run(Epi&& epi) {
+    const int items = p.RG * p.chunks_per_row * p.nsets;
+    const int beg = static_cast<int>(static_cast<long long>(blockIdx.x) * items / gridDim.x);
+    const int end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * items / gridDim.x);
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) {
+      for (int i = 0; i < nstage; ++i) {
+        mbar_init(&full[i], 1);
+        mbar_init(&empty[i], kScanConsumerWarps);
+      }
+      *abort_flag = 0;
+      asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    __syncthreads();
+    if (warp == kScanConsumerWarps) {
+      produce(beg, end);
+      return;
+    }
+    int cur_u = -1;
+    float acc[32];
+    for (int it = beg; it < end; ++it) {
+      const int k = it - beg, st = k % nstage;
+      int u, c, s;
+      decode_item(it, u, c, s);
+      if (u != cur_u) {
+        consumer_sync();
+        build_tables(u);
+        consumer_sync();
+        cur_u = u;
+      }
+      if (!mbar_wait(&full[st], (k / nstage) & 1)) {
+        fail_timeout();
+        return;
+      }
+      const int nr = p.n[u / p.Gheads];
+      const int w0 = c * kChunkWords;
+      if (s == 0) {
+        const float C = p.C[u];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] = C;
+      }
+      if (32 * w0 < nr) compute_set(p.nsets * TBL_BYTES + st * STAGE_BYTES, s, acc);
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[st]);
+      if (s == p.nsets - 1) epi(u, w0, nr, acc, static_cast<int>(threadIdx.x));
+    }
+  }
+};
+
+}  // namespace kvs

@@ -1,0 +1,260 @@
+"""GPU parity of the Fathom path against the CPU oracle, through the C ABI.
+
+Integer work (index codes, bit allocation, top-k on identical scores, slots,
+misses) is compared bit for bit; float work within the tolerances of
+tests/_parity.py. Sizes span several tiles and a ragged tail.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests._parity import ATTN_TOL, check_selection, fathom_score_tol
+
+pytestmark = pytest.mark.gpu
+D = 128
+
+
+@pytest.fixture(scope="module")
+def kvs():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import kv_index_scan_b200
+    return kv_index_scan_b200
+
+
+DEV = "cuda"
+
+
+def _np(t):
+    t = t.detach().cpu()
+    if t.dtype == torch.bfloat16:
+        t = t.view(torch.int16)
+    return t.numpy()
+
+
+# ----------------------------------------------------------------------------- a0 index
+
+@pytest.mark.parametrize("R,G,nl,n_max", [(1, 1, [4096], 4096), (2, 3, [1000, 33], 1030),
+                                          (1, 2, [32], 32), (2, 1, [0, 5000], 5000)])
+def test_index_build_bit_exact(kvs, R, G, nl, n_max):
+    K, _, _ = synth.fathom_kv(R, G, D, nl, n_max=n_max, seed=21, with_v=False)
+    W = kvs.plane_words(n_max)
+    ix = kvs.build_fathom_index(K.to(DEV), nl, W)
+    torch.cuda.synchronize()
+    planes, kmin, kstep, kvar = oracle.build_index_batch(K, nl, W)
+    assert np.array_equal(_np(ix.planes).view(np.uint32), planes)
+    assert np.array_equal(_np(ix.kmin), kmin)
+    assert np.array_equal(_np(ix.kstep), kstep)
+    assert np.array_equal(_np(ix.kvar), kvar)
+
+
+# ----------------------------------------------------------------------------- a1 allocation
+
+@pytest.mark.parametrize("B", [0, 1, 4, 68, 92, 136, 511, 512])
+def test_plan_bits_bit_exact(kvs, B):
+    R, G, H, n = 2, 4, 4, 3000
+    K, _, nl = synth.fathom_kv(R, G, D, n, seed=B + 1, with_v=False)
+    q = synth.queries(R, G, H, D, seed=B + 1)
+    ix = kvs.build_fathom_index(K.to(DEV), nl)
+    plan = kvs.fathom_plan_bits(q.to(DEV), ix, B)
+    torch.cuda.synchronize()
+    kvar, kmin, kstep = _np(ix.kvar), _np(ix.kmin), _np(ix.kstep)
+    t_gpu = _np(plan.t)
+    for r in range(R):
+        for g in range(G):
+            t, qbar = oracle.plan_bits(q[r, g], kvar[r, g], B)
+            assert np.array_equal(t_gpu[r, g], t)
+            if B == 0:
+                continue
+            pidx = _np(plan.plane_idx)[r, g, :B].view(np.uint16).astype(np.int64)
+            exp = np.array([4 * c + p for c in range(D) for p in range(t[c])], np.int64)
+            assert np.array_equal(pidx, exp)
+            c, p = exp // 4, exp % 4
+            wref = qbar[c].astype(np.float64) * kstep[r, g][c].astype(np.float64) * 2.0 ** (3 - p)
+            assert np.allclose(_np(plan.plane_w)[r, g, :B], wref, rtol=2 ** -23, atol=0)
+            cref = np.sum(qbar.astype(np.float64) * (kmin[r, g].astype(np.float64) + kstep[r, g].astype(np.float64)
+                                                     * (2.0 ** (4 - t.astype(np.float64)) - 1) / 2))
+            tol = fathom_score_tol(qbar, kmin[r, g], kstep[r, g], 0)
+            assert abs(float(_np(plan.C)[r, g]) - cref) <= tol
+
+
+# ----------------------------------------------------------------------------- a2 scan
+
+@pytest.mark.parametrize("B", [0, 68, 92, 136, 512])
+@pytest.mark.parametrize("nl,n_max", [([4096, 4095], 4096), ([33, 1], 64), ([20000, 12345], 20000)])
+def test_fathom_scan_within_f32_error(kvs, B, nl, n_max):
+    R, G, H = 2, 2, 4
+    K, _, _ = synth.fathom_kv(R, G, D, nl, n_max=n_max, seed=7, with_v=False)
+    q = synth.queries(R, G, H, D, seed=7)
+    ix = kvs.build_fathom_index(K.to(DEV), nl)
+    plan = kvs.fathom_plan_bits(q.to(DEV), ix, B)
+    sc = kvs.index_scan_fathom(ix, plan, nl, n_max)
+    torch.cuda.synchronize()
+    sc = _np(sc)
+    planes, kmin, kstep, kvar = (_np(ix.planes).view(np.uint32), _np(ix.kmin), _np(ix.kstep), _np(ix.kvar))
+    for r in range(R):
+        for g in range(G):
+            t, qbar = oracle.plan_bits(q[r, g], kvar[r, g], B)
+            ref = oracle.scan(planes[r, g], kmin[r, g], kstep[r, g], qbar, t, nl[r])
+            tol = fathom_score_tol(qbar, kmin[r, g], kstep[r, g], B)
+            assert np.max(np.abs(sc[r, g, : nl[r]] - ref), initial=0) <= tol
+            assert np.all(np.isneginf(sc[r, g, nl[r]:]))
+
+
+# ----------------------------------------------------------------------------- a3 top-k
+
+@pytest.mark.parametrize("n,k", [(1, 1), (100, 7), (4096, 256), (4097, 2048), (131072, 2048),
+                                 (70000, 3000), (50, 64)])
+def test_topk_bit_exact_on_identical_scores(kvs, n, k):
+    rng = np.random.default_rng(n + k)
+    R, G = 2, 3
+    nl = [n, max(1, n // 3)]
+    s = np.round(rng.standard_normal((R, G, n)) * 50).astype(np.float32)  # many ties
+    s[:, :, ::97] = s[:, :, 0:1]  # more exact ties
+    st = torch.from_numpy(s).to(DEV)
+    idx, vals = kvs.topk_select(st, nl, k, want_vals=True)
+    torch.cuda.synchronize()
+    idx, vals = _np(idx), _np(vals)
+    for r in range(R):
+        for g in range(G):
+            ref, ke = oracle.topk(s[r, g, : nl[r]].copy(), k)
+            assert np.array_equal(idx[r, g], ref)
+            assert np.array_equal(vals[r, g, :ke], s[r, g][ref[:ke]])
+            assert np.all(np.isneginf(vals[r, g, ke:]))
+
+
+@pytest.mark.parametrize("n,block,k", [(80000, 64, 2048), (1000, 64, 256), (4096, 32, 2048),
+                                       (100, 64, 2048)])
+def test_block_topk_bit_exact(kvs, n, block, k):
+    rng = np.random.default_rng(n)
+    R = 3
+    nl = [n, n - 17, max(1, n // 5)]
+    nb = (n + block - 1) // block
+    s = np.round(rng.standard_normal((R, nb)) * 20).astype(np.float32)
+    idx = _np(kvs.topk_select(torch.from_numpy(s).to(DEV), nl, k, block=block))
+    for r in range(R):
+        nbr = (nl[r] + block - 1) // block
+        ref, cnt = oracle.block_topk(s[r, :nbr].copy(), nl[r], block, k)
+        assert np.array_equal(idx[r], ref)
+
+
+# ----------------------------------------------------------------------------- a4 gather
+
+def test_gather_bit_exact(kvs):
+    R, G, n, k, S = 2, 3, 5000, 512, 1024
+    K, V, nl = synth.fathom_kv(R, G, D, [n, 3000], n_max=n, seed=5)
+    rng = np.random.default_rng(0)
+    sel = np.full((R, G, k), -1, np.int32)
+    for r in range(R):
+        for g in range(G):
+            kk = k if r == 0 else k - 100  # ragged selections with -1 padding
+            sel[r, g, :kk] = np.sort(rng.choice(nl[r], kk, replace=False))
+    slot_map, hot_tok = synth.slot_map_from_selection(sel, nl, n, S, 0.2, seed=5)
+    hotK, hotV = synth.hot_rows(K, hot_tok), synth.hot_rows(V, hot_tok)
+    gK, gV, slots, misses = kvs.sparse_gather(torch.from_numpy(sel).to(DEV),
+                                              torch.from_numpy(slot_map).to(DEV), hotK.to(DEV),
+                                              hotV.to(DEV), K.to(DEV), V.to(DEV), nl)
+    torch.cuda.synchronize()
+    for r in range(R):
+        for g in range(G):
+            rK, rV, rs, rm = oracle.gather(sel[r, g], slot_map[r, g], hotK[r, g], hotV[r, g], K[r, g], V[r, g])
+            assert np.array_equal(_np(gK[r, g]).view(np.uint16), rK)
+            assert np.array_equal(_np(gV[r, g]).view(np.uint16), rV)
+            assert np.array_equal(_np(slots[r, g]), rs)
+            assert int(misses[r, g]) == rm
+
+
+# ----------------------------------------------------------------------------- a5 attention
+
+@pytest.mark.parametrize("H", [1, 4, 8])
+@pytest.mark.parametrize("k", [1, 64, 100, 2048])
+@pytest.mark.parametrize("qdt", [torch.float32, torch.bfloat16])
+def test_attention_within_tolerance(kvs, H, k, qdt):
+    R, G = 2, 3
+    K, V, _ = synth.fathom_kv(R, G, D, k, seed=H + k)
+    q = synth.queries(R, G, H, D, seed=H + k, dtype=qdt)
+    k_eff = torch.tensor([[k, max(1, k // 2), 0], [k, 1, k]], dtype=torch.int32)
+    out, lse = kvs.sparse_decode_attn(q.to(DEV), K.to(DEV), V.to(DEV), k_eff.to(DEV))
+    torch.cuda.synchronize()
+    out, lse = _np(out), _np(lse)
+    for r in range(R):
+        for g in range(G):
+            ke = int(k_eff[r, g])
+            ro, rl = oracle.attention(q[r, g].float(), K[r, g], V[r, g], ke, 1 / math.sqrt(D))
+            assert np.max(np.abs(out[r, g] - ro)) < ATTN_TOL
+            if ke:
+                assert np.max(np.abs(lse[r, g] - rl)) < 1e-3
+            else:
+                assert np.all(np.isneginf(lse[r, g])) and not out[r, g].any()
+
+
+# ----------------------------------------------------------------------------- a6 decode step
+
+def _decode_case(kvs, R, G, H, nl, n_max, B, k, S, seed, rows=None):
+    K, V, _ = synth.fathom_kv(R, G, D, nl, n_max=n_max, seed=seed)
+    q = synth.queries(R, G, H, D, seed=seed)
+    W = kvs.plane_words(n_max)
+    planes, kmin, kstep, kvar = oracle.build_index_batch(K, nl, W)
+    scale = 1 / math.sqrt(D)
+    ref0 = oracle.decode_batch(q, planes, kmin, kstep, kvar, nl, B, k, None, None, None, K, V, scale,
+                               rows=rows)
+    slot_map, hot_tok = synth.slot_map_from_selection(ref0["idx"], nl, n_max, S, 0.2, seed=seed)
+    hotK, hotV = synth.hot_rows(K, hot_tok), synth.hot_rows(V, hot_tok)
+    ref = oracle.decode_batch(q, planes, kmin, kstep, kvar, nl, B, k, slot_map, hotK, hotV, K, V,
+                              scale, rows=rows, want_scores=True)
+    ix = kvs.build_fathom_index(K.to(DEV), nl, W)
+    step = kvs.DecodeStep(ix, nl, n_max, H, B, k, K.to(DEV), V.to(DEV),
+                          torch.from_numpy(slot_map).to(DEV), hotK.to(DEV), hotV.to(DEV))
+    step(q.to(DEV))
+    torch.cuda.synchronize()
+    return ref, step
+
+
+def _check_decode(ref, step, R, G, nl, k, rows=None):
+    t, idx, slots, misses = _np(step.plan.t), _np(step.idx), _np(step.slots), _np(step.misses)
+    out, lse = _np(step.out), _np(step.lse)
+    rows = range(R * G) if rows is None else rows
+    diffs = 0
+    for u in rows:
+        r, g = divmod(u, G)
+        ke = min(k, nl[r])
+        assert np.array_equal(t[r, g], ref["t"][r, g])
+        d = check_selection(idx[r, g], ref["idx"][r, g], ref["scores"][r, g, : nl[r]], ke)
+        diffs += d
+        if d == 0:
+            assert np.array_equal(slots[r, g], ref["slots"][r, g])
+            assert misses[r, g] == ref["misses"][r, g]
+            assert np.max(np.abs(out[r, g] - ref["out"][r, g])) < ATTN_TOL
+            assert np.max(np.abs(lse[r, g] - ref["lse"][r, g])) < 1e-3
+    return diffs
+
+
+def test_decode_step_tiny_config(kvs):
+    """1 request, 1 KV head of 4 query heads, 4096 keys, B = 92, top-256, 512 slots at 80% hits."""
+    ref, step = _decode_case(kvs, 1, 1, 4, [4096], 4096, 92, 256, 512, seed=0)
+    assert _check_decode(ref, step, 1, 1, [4096], 256) == 0
+    assert int(step.misses[0, 0]) == round(0.2 * 256)
+
+
+@pytest.mark.parametrize("B", [68, 92, 136, 512])
+def test_decode_step_ragged_batch(kvs, B):
+    nl = [20000, 7777, 2048, 1000]
+    ref, step = _decode_case(kvs, 4, 2, 4, nl, 20000, B, 2048, 4096, seed=B)
+    _check_decode(ref, step, 4, 2, nl, 2048)
+
+
+def test_decode_step_layer_sharing_reuses_selection(kvs):
+    """idx_in: the second layer of a group reads the first layer's selection."""
+    nl = [6000, 5000]
+    ref, step = _decode_case(kvs, 2, 2, 4, nl, 6000, 92, 512, 1024, seed=3)
+    out1 = step.out.clone()
+    idx = step.idx.clone()
+    step.idx.fill_(-7)
+    step(step_q := synth.queries(2, 2, 4, D, seed=3).to(DEV), idx_in=idx)
+    torch.cuda.synchronize()
+    assert torch.all(step.idx == -7)  # not written when a selection is given
+    assert torch.equal(step.out, out1)
