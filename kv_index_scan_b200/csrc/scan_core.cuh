@@ -303,9 +303,11 @@ struct ScanCore {
   // called by every consumer thread at the end of each chunk.
   template <typename Epi>
   __device__ void run(Epi&& epi) {
-    const int items = p.RG * p.chunks_per_row * p.nsets;
-    const int beg = static_cast<int>(static_cast<long long>(blockIdx.x) * items / gridDim.x);
-    const int end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * items / gridDim.x);
+    // whole chunks per block: the sets of a chunk accumulate in one thread
+    const int chunks = p.RG * p.chunks_per_row;
+    const int cbeg = static_cast<int>(static_cast<long long>(blockIdx.x) * chunks / gridDim.x);
+    const int cend = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * chunks / gridDim.x);
+    const int beg = cbeg * p.nsets, end = cend * p.nsets;
     const int warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) {
       for (int i = 0; i < nstage; ++i) {
@@ -320,7 +322,11 @@ struct ScanCore {
       produce(beg, end);
       return;
     }
+    // Consumers never leave early: after a timed-out wait they stop working
+    // but keep stepping through the same items, so that every named barrier
+    // below is still met by all of them.
     int cur_u = -1;
+    bool dead = false;
     float acc[32];
     for (int it = beg; it < end; ++it) {
       const int k = it - beg, st = k % nstage;
@@ -328,13 +334,15 @@ struct ScanCore {
       decode_item(it, u, c, s);
       if (u != cur_u) {
         consumer_sync();
-        build_tables(u);
+        if (!dead) build_tables(u);
         consumer_sync();
         cur_u = u;
       }
+      if (dead) continue;
       if (!mbar_wait(&full[st], (k / nstage) & 1)) {
         fail_timeout();
-        return;
+        dead = true;
+        continue;
       }
       const int nr = p.n[u / p.Gheads];
       const int w0 = c * kChunkWords;

@@ -72,9 +72,9 @@ kvs_status launch_gb(const ScanParams& p, cudaStream_t s) {
   const size_t smem = ScanCore<G, b>::smem_bytes(p.nsets);
   auto kern = fathom_scan_lut_kernel<G, b>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  const int items = p.RG * p.chunks_per_row * p.nsets;
-  if (items <= 0) return KVS_OK;
-  const int grid = min(items, sm_count());
+  const int chunks = p.RG * p.chunks_per_row;
+  if (chunks <= 0) return KVS_OK;
+  const int grid = min(chunks, sm_count());
   kern<<<grid, kScanThreads, smem, s>>>(p);
   return check_launch("index_scan(fathom, lut)");
 }

@@ -84,8 +84,9 @@ def test_plan_bits_bit_exact(kvs, B):
 
 # ----------------------------------------------------------------------------- a2 scan
 
-@pytest.mark.parametrize("B", [0, 68, 92, 136, 512])
-@pytest.mark.parametrize("nl,n_max", [([4096, 4095], 4096), ([33, 1], 64), ([20000, 12345], 20000)])
+@pytest.mark.parametrize("B", [0, 1, 7, 33, 68, 72, 73, 92, 136, 144, 145, 300, 512])
+@pytest.mark.parametrize("nl,n_max", [([4096, 4095], 4096), ([33, 1], 64), ([20000, 12345], 20000),
+                                      ([0, 70000], 70001)])
 def test_fathom_scan_within_f32_error(kvs, B, nl, n_max):
     R, G, H = 2, 2, 4
     K, _, _ = synth.fathom_kv(R, G, D, nl, n_max=n_max, seed=7, with_v=False)
