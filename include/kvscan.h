@@ -258,6 +258,31 @@ KVS_API kvs_status sparse_decode_attn(const void* q, int32_t q_dtype, const uint
                               void* stream);
 KVS_API size_t kvs_attn_workspace_size(int32_t R, int32_t G, int32_t H, int32_t k);
 
+/* sparse_decode_attn_noalloc: the same computation as sparse_decode_attn
+ * (same arguments except that there is no workspace), for callers that cannot
+ * allocate device memory: code that runs where cudaMalloc is not allowed or
+ * would stall the device (inside a stream being captured into a CUDA graph,
+ * allocator-free runtimes that hand the library only their input and output
+ * buffers, or latency-critical serving loops that forbid allocation after
+ * start-up). The pages have no counterpart: this is a library convenience.
+ *
+ * Its scratch (the split-K partial results) is one fixed 4 MiB device array
+ * inside this library, which every GPU that loads the library holds until the
+ * process exits. The need is kvs_attn_workspace_size() and stays below
+ * 8 * (SM count) * H * 528 bytes; on a 148-SM B200 every size with H <= 4
+ * fits. Sizes that need more are rejected with KVS_EINVAL and a message. The call allocates nothing and calls no
+ * allocator. The first call on each device looks up that device's address of
+ * the array (with the device current); make that first call before any
+ * stream capture. Every call shares the array: nothing in it has to start at
+ * zero (each split writes its whole partial before the merge reads it), but
+ * calls that overlap on the same GPU (other streams, other host threads)
+ * race on it and must be serialised by the caller. */
+KVS_API kvs_status sparse_decode_attn_noalloc(const void* q, int32_t q_dtype, const uint16_t* K,
+                                              const uint16_t* V, const int32_t* k_eff, int32_t R,
+                                              int32_t G, int32_t H, int32_t D, int32_t k,
+                                              float scale, float* out, float* lse,
+                                              int32_t* dev_status, void* stream);
+
 /* ---------------------------------------------------------------------------
  * a6: one fused decode step for all (r, g), on one stream.
  *

@@ -84,6 +84,8 @@ def _declare():
     L.sparse_decode_attn.restype = I32
     L.kvs_attn_workspace_size.argtypes = [I32, I32, I32, I32]
     L.kvs_attn_workspace_size.restype = SZ
+    L.sparse_decode_attn_noalloc.argtypes = [P, I32, P, P, P, I32, I32, I32, I32, I32, F32, P, P, P, P]
+    L.sparse_decode_attn_noalloc.restype = I32
     L.decode_step.argtypes = [ctypes.POINTER(DecodeArgsC), P, SZ, P, P]
     L.decode_step.restype = I32
     L.kvs_decode_step_workspace_size.argtypes = [I32, I32, I32, I32, I32, I32]
@@ -293,6 +295,21 @@ def sparse_decode_attn(q, K, V, k_eff=None, scale: float | None = None, want_lse
                                  H, D, k, scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                  _ptr(dev_status), _stream(stream))
     _check(st, "sparse_decode_attn")
+    return out, lse
+
+
+def sparse_decode_attn_noalloc(q, K, V, out, lse=None, k_eff=None, scale: float | None = None,
+                               stream=None, dev_status=None):
+    """a5 without a workspace, into caller-provided out (and lse): the library
+    keeps the split-K scratch in a fixed device array (see include/kvscan.h)."""
+    R, G, H, D = q.shape
+    k = K.shape[2]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    qd = KVS_BF16 if q.dtype == torch.bfloat16 else KVS_F32
+    st = _lib.sparse_decode_attn_noalloc(_ptr(_u16(q)), qd, _ptr(_u16(K)), _ptr(_u16(V)), _ptr(k_eff),
+                                         R, G, H, D, k, scale, _ptr(out), _ptr(lse),
+                                         _ptr(dev_status), _stream(stream))
+    _check(st, "sparse_decode_attn_noalloc")
     return out, lse
 
 

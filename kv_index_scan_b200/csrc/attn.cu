@@ -318,3 +318,81 @@ kvs_status attn_launch(const void* q, int q_bf16, const RowSrc& src, int RG, int
 }
 
 }  // namespace kvs
+
+// ----------------------------------------------------------------------------
+// sparse_decode_attn_noalloc: the same attention for callers that cannot
+// allocate device memory. Its split-K partial results (the only scratch the
+// attention needs) live in one fixed array of this library instead of a
+// caller workspace.
+#include <mutex>
+
+namespace {
+
+// 4 MiB of partial results (R*G*nsplit*H*(128+4) floats). The split count
+// falls as the batch grows (about 4 blocks per SM in all), so the need stays
+// below 8 * SMs * H * 528 bytes: on a 148-SM B200 every size with H <= 4 fits,
+// and only H >= 7 with a few hundred (request, KV head) rows exceeds it.
+// Every GPU that loads this library holds the array until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) float g_attn_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+std::mutex g_scratch_mu;
+float* g_scratch_dev[64] = {nullptr};
+
+// Device address of g_attn_scratch on the current device. The name of the
+// array in host code is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+kvs_status noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return kvs::fail(KVS_ECUDA, "sparse_decode_attn_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return kvs::fail(KVS_EUNSUPPORTED, "sparse_decode_attn_noalloc: device %d", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_dev[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_attn_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return kvs::fail(KVS_ECUDA, "sparse_decode_attn_noalloc: cudaGetSymbolAddress: %s",
+                       cudaGetErrorString(e));
+    g_scratch_dev[dev] = static_cast<float*>(p);
+  }
+  *out = g_scratch_dev[dev];
+  return KVS_OK;
+}
+
+}  // namespace
+
+extern "C" kvs_status sparse_decode_attn_noalloc(const void* q, int32_t q_dtype, const uint16_t* K,
+                                                 const uint16_t* V, const int32_t* k_eff, int32_t R,
+                                                 int32_t G, int32_t H, int32_t D, int32_t k,
+                                                 float scale, float* out, float* lse,
+                                                 int32_t* dev_status, void* stream) {
+  using namespace kvs;
+  (void)dev_status;
+  KVS_REQUIRE(q && K && V && out, KVS_EINVAL, "sparse_decode_attn_noalloc: null pointer argument");
+  KVS_REQUIRE(q_dtype == KVS_F32 || q_dtype == KVS_BF16, KVS_EINVAL,
+              "sparse_decode_attn_noalloc: q_dtype=%d", q_dtype);
+  KVS_REQUIRE(R >= 1 && G >= 1 && k >= 1 && H >= 1 && H <= 8, KVS_EINVAL,
+              "sparse_decode_attn_noalloc: R=%d G=%d H=%d k=%d", R, G, H, k);
+  KVS_REQUIRE(D == kD, KVS_EUNSUPPORTED, "sparse_decode_attn_noalloc: D=%d (only 128 is built)", D);
+  KVS_REQUIRE(aligned16(K) && aligned16(V) && aligned16(out), KVS_EINVAL,
+              "sparse_decode_attn_noalloc: K, V and out must be 16-byte aligned");
+  const size_t need = attn_ws_bytes(R * G, H, k);
+  KVS_REQUIRE(need <= kNoAllocScratchBytes, KVS_EINVAL,
+              "sparse_decode_attn_noalloc: R=%d G=%d H=%d k=%d needs %zu bytes of scratch, more "
+              "than the fixed %zu-byte array; use sparse_decode_attn with a workspace",
+              R, G, H, k, need, kNoAllocScratchBytes);
+  float* scratch = nullptr;
+  kvs_status st = noalloc_scratch(&scratch);
+  if (st != KVS_OK) return st;
+  RowSrc src{};
+  src.mode = kRowsStaged;
+  src.K = K;
+  src.V = V;
+  src.k_eff = k_eff;
+  src.G = G;
+  src.k = k;
+  st = attn_launch(q, q_dtype == KVS_BF16, src, R * G, H, scale, out, lse, scratch,
+                   static_cast<cudaStream_t>(stream));
+  return st == KVS_OK ? ok() : st;
+}
