@@ -79,49 +79,76 @@ def _max_over_ranks(dist, x: float) -> float:
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """SM clock and throttle-reason samples taken every 10 ms by an NVML thread
+    while the timed region runs (nvidia-smi is the fallback). The sampler is
+    started before the region and must have one sample under load before the
+    region starts."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self):
-        self.proc = None
-        self.path = None
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = False
+        self._thread = None
+        self._nvml = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(torch.cuda.current_device())
+        bus = getattr(props, "pci_bus_id", None)
+        dom = getattr(props, "pci_domain_id", 0)
+        dev = getattr(props, "pci_device_id", 0)
+        if bus is not None:
+            try:
+                return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{bus:02x}:{dev:02x}.0")
+            except Exception:
+                pass
+        idx = int((os.environ.get("CUDA_VISIBLE_DEVICES", "") or str(torch.cuda.current_device())).split(",")[0])
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(idx)
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
-        dev = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0] or str(torch.cuda.current_device())
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        import threading
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={dev}", f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except (FileNotFoundError, OSError):
-            self.proc = None
+            nv, h = self._handle()
+        except Exception as e:  # no NVML
+            self.reasons.add(f"nvml unavailable: {type(e).__name__}")
+            return
+        self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+
+        def loop():
+            while not self._stop:
+                try:
+                    self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    r = (nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                         if hasattr(nv, "nvmlDeviceGetCurrentClocksEventReasons")
+                         else nv.nvmlDeviceGetCurrentClocksThrottleReasons(h))
+                    for name, bit in self.REASONS.items():
+                        if r & bit:
+                            self.reasons.add(name)
+                except Exception:
+                    pass
+                time.sleep(0.01)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+
+    def wait_first(self, timeout=2.0):
+        t0 = time.time()
+        while self._thread is not None and not self.samples and time.time() - t0 < timeout:
+            time.sleep(0.005)
+        self.samples.clear()
 
     def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        self.proc.wait()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    smax = float(parts[2])
-                except ValueError:
-                    continue
-                for nm, v in zip(names, parts[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(nm)
-        os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        self._stop = True
+        if self._thread is not None:
+            self._thread.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
 
 
 def setup(cfg: dict, device, seed: int = 1):
@@ -183,6 +210,7 @@ def run_ours(args, cfg, dist, rank, ws):
     torch.cuda.synchronize()
     clocks = Clocks()
     clocks.start()
+    clocks.wait_first()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
@@ -260,7 +288,7 @@ def step_needs_combine(cfg) -> bool:
     return kvs._lib.kvs_attn_workspace_size(cfg["R"], cfg["G"], cfg["H"], cfg["k"]) > 0
 
 
-def cpu_baseline(cfg, data, rows: int = 8) -> dict:
+def cpu_baseline(cfg, data, rows: int = 8, min_seconds: float = 10.0) -> dict:
     """The CPU oracle, as it stands, on a bounded sample of the same workload:
     `rows` (request, KV head) rows of the decode step, all host cores."""
     import oracle
@@ -279,13 +307,18 @@ def cpu_baseline(cfg, data, rows: int = 8) -> dict:
     W = synth.plane_words(n)
     planes, kmin, kstep, kvar = oracle.build_index_batch(K, nl, W)  # data prep, not timed
     cores = os.cpu_count() or 1
-    t0 = time.perf_counter()
-    oracle.decode_batch(q, planes, kmin, kstep, kvar, nl, B, k, sm, hK, hV, K, V,
-                        1 / math.sqrt(128), nthreads=cores)
-    dt = time.perf_counter() - t0
-    return {"value": rows * n / dt, "unit": "keys/s", "cores": cores, "kind": "oracle",
+    reps, t0 = 0, time.perf_counter()
+    while True:  # repeat the bounded sample until ~10 s of CPU work
+        oracle.decode_batch(q, planes, kmin, kstep, kvar, nl, B, k, sm, hK, hV, K, V,
+                            1 / math.sqrt(128), nthreads=cores)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_seconds or reps >= 200:
+            break
+    return {"value": reps * rows * n / dt, "unit": "keys/s", "cores": cores, "kind": "oracle",
             "sample": f"{rows} of {R * G} (request, KV head) rows of one decode step "
-                      f"({rows * n} keys), fp64 C++ oracle, {dt:.2f} s"}
+                      f"({rows * n} keys) x {reps} repetitions, fp64 C++ oracle on {cores} "
+                      f"threads, {dt:.1f} s"}
 
 
 def run_reference(args, cfg, dist, rank, ws):
@@ -331,7 +364,7 @@ def run_reference(args, cfg, dist, rank, ws):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="qwen3-8b-128k", choices=sorted(WORKLOADS))

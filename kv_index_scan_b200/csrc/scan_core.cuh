@@ -8,9 +8,10 @@
 
 namespace kvs {
 
-constexpr int kScanConsumerWarps = 4;
+constexpr int kScanConsumerWarps = 8;
 constexpr int kScanThreads = 32 * (kScanConsumerWarps + 1);  // + one producer warp
-constexpr int kChunkWords = 32 * kScanConsumerWarps;          // one 32-key word per consumer thread
+constexpr int kKeysPerThread = 16;                            // half of a 32-key word
+constexpr int kChunkWords = 16 * kScanConsumerWarps;          // two consumer threads per word
 constexpr int kRowBytes = 4 * kChunkWords;                    // 512 bytes of a plane per chunk
 constexpr long long kWaitCycles = 2000000000ll;               // ~1 s bound on every wait
 
@@ -109,39 +110,35 @@ __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;\n" ::"n"(32 * kScanConsumerWarps) : "memory");
 }
 
-// 32x32 bit transpose in registers: afterwards bit c of x[r] is bit r of the
-// original x[c]. Byte-level stages with byte permutes, bit-level stages with
-// a shift and a bit select each.
-__device__ __forceinline__ void transpose32(uint32_t (&x)[32]) {
+// Half of a 32x32 bit transpose, in registers. On entry x[k] holds, for one
+// 16-key half of a word, the 16 bits of plane k in its low half and those of
+// plane k + 16 in its high half (the first, 16-bit stage of the full
+// transpose, done by the loads). On exit bit c of x[r] is plane c's bit for
+// key r of the half. One byte-permute stage and three shift/select stages.
+__device__ __forceinline__ void transpose16(uint32_t (&x)[16]) {
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
-    const uint32_t a = x[k], c = x[k + 16];
-    x[k] = __byte_perm(a, c, 0x5410);
-    x[k + 16] = __byte_perm(a, c, 0x7632);
-  }
-#pragma unroll
-  for (int k = 0; k < 32; ++k) {
     if (k & 8) continue;
     const uint32_t a = x[k], c = x[k + 8];
     x[k] = __byte_perm(a, c, 0x6240);
     x[k + 8] = __byte_perm(a, c, 0x7351);
   }
 #pragma unroll
-  for (int k = 0; k < 32; ++k) {
+  for (int k = 0; k < 16; ++k) {
     if (k & 4) continue;
     const uint32_t t = ((x[k] >> 4) ^ x[k + 4]) & 0x0F0F0F0Fu;
     x[k + 4] ^= t;
     x[k] ^= t << 4;
   }
 #pragma unroll
-  for (int k = 0; k < 32; ++k) {
+  for (int k = 0; k < 16; ++k) {
     if (k & 2) continue;
     const uint32_t t = ((x[k] >> 2) ^ x[k + 2]) & 0x33333333u;
     x[k + 2] ^= t;
     x[k] ^= t << 2;
   }
 #pragma unroll
-  for (int k = 0; k < 32; ++k) {
+  for (int k = 0; k < 16; ++k) {
     if (k & 1) continue;
     const uint32_t t = ((x[k] >> 1) ^ x[k + 1]) & 0x55555555u;
     x[k + 1] ^= t;
@@ -248,30 +245,38 @@ struct ScanCore {
     }
   }
 
-  // The set's contribution for this thread's 32 keys, added into acc.
-  __device__ __forceinline__ void compute_set(int stage_off, int s, float (&acc)[32]) const {
+  // Offset of stream position o (a static plane slot of the set) for a lane
+  // whose planes are rotated by lp groups.
+  __device__ __forceinline__ static int slot_offset(int o, int lp) {
+    const int g = o / b, bi = o % b;
+    return (((g + lp) & (G - 1)) * b + bi) * kRowBytes;
+  }
+
+  // The set's contribution for this thread's 16 keys, added into acc. Thread
+  // t handles half (t & 1) of word (t >> 1) of the chunk: it reads that 16-bit
+  // half of each plane word and transposes a 32-plane x 16-key block.
+  __device__ __forceinline__ void compute_set(int stage_off, int s, float (&acc)[kKeysPerThread]) const {
+    constexpr int NK = kKeysPerThread;
     const int t = threadIdx.x;
     const int lane = t & 31;
     const int lp = lane % G, repl = lane / G;
-    const unsigned char* mine = g_scan_smem + stage_off + 4 * t;
-    uint32_t prev[32];
+    const unsigned char* mine = g_scan_smem + stage_off + 4 * (t >> 1) + 2 * (t & 1);
+    uint32_t prev[NK];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) prev[j] = 0u;
+    for (int j = 0; j < NK; ++j) prev[j] = 0u;
 #pragma unroll
     for (int m = 0; m < NBLK; ++m) {
-      uint32_t x[32];
+      uint32_t x[NK];
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        const int o = 32 * m + q;
-        if (o < NPOS) {
-          const int g = o / b, bi = o % b;
-          const int gr = (g + lp) & (G - 1);
-          x[q] = *reinterpret_cast<const uint32_t*>(mine + (gr * b + bi) * kRowBytes);
-        } else {
-          x[q] = 0u;
-        }
+      for (int q = 0; q < NK; ++q) {
+        const int o1 = 32 * m + q, o2 = o1 + 16;
+        const uint32_t lo =
+            o1 < NPOS ? *reinterpret_cast<const uint16_t*>(mine + slot_offset(o1, lp)) : 0u;
+        const uint32_t hi =
+            o2 < NPOS ? *reinterpret_cast<const uint16_t*>(mine + slot_offset(o2, lp)) : 0u;
+        x[q] = __byte_perm(lo, hi, 0x5410);
       }
-      transpose32(x);
+      transpose16(x);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const int st = g * b, en = st + b - 1;
@@ -282,7 +287,7 @@ struct ScanCore {
                                                   s * TBL_BYTES);
         constexpr uint32_t mask7 = ((1u << b) - 1u) << 7;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < NK; ++j) {
           uint32_t v;
           if (straddle)
             v = __funnelshift_r(prev[j], x[j], sh - 7);
@@ -295,7 +300,7 @@ struct ScanCore {
         }
       }
 #pragma unroll
-      for (int j = 0; j < 32; ++j) prev[j] = x[j];
+      for (int j = 0; j < NK; ++j) prev[j] = x[j];
     }
   }
 
@@ -327,7 +332,7 @@ struct ScanCore {
     // below is still met by all of them.
     int cur_u = -1;
     bool dead = false;
-    float acc[32];
+    float acc[kKeysPerThread];
     for (int it = beg; it < end; ++it) {
       const int k = it - beg, st = k % nstage;
       int u, c, s;
@@ -349,7 +354,7 @@ struct ScanCore {
       if (s == 0) {
         const float C = p.C[u];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) acc[j] = C;
+        for (int j = 0; j < kKeysPerThread; ++j) acc[j] = C;
       }
       if (32 * w0 < nr) compute_set(p.nsets * TBL_BYTES + st * STAGE_BYTES, s, acc);
       __syncwarp();

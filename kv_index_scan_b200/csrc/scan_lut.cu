@@ -15,11 +15,12 @@
 //    memory stage with 1-D TMA bulk copies (cp.async.bulk, 512 bytes per
 //    plane), completing on the stage's mbarrier. Stages form a ring; consumer
 //    warps release a stage when done with it. Every wait is bounded.
-//  * Transpose. A consumer thread owns one 32-key word. It loads 32 plane
-//    words (one per plane, conflict-free 4-byte reads) and transposes the
-//    32x32 bit matrix in registers (two byte-permute stages, three
-//    shift/select stages: ~0.25 operations per bit), giving per key a word of
-//    32 plane bits.
+//  * Transpose. Two consumer threads share a 32-key word, 16 keys each. A
+//    thread loads its 16-bit half of 32 plane words (conflict-free 2-byte
+//    reads), pairs planes k and k + 16 in one register, and finishes the
+//    32-plane x 16-key bit transpose in registers (one byte-permute stage,
+//    three shift/select stages: ~0.25 operations per bit), giving per key a
+//    word of 32 plane bits.
 //  * Lookup. The planes are cut into G groups (8 or 16) of b bits (b <= 9);
 //    group g has a 2^b-entry table of the sums of its weights. One lookup per
 //    key per group replaces b multiply-adds. To keep the 32 lanes of a warp
@@ -42,16 +43,15 @@ namespace {
 template <int G, int b>
 __global__ void __launch_bounds__(kScanThreads, 1) fathom_scan_lut_kernel(ScanParams p) {
   ScanCore<G, b> core(p);
-  core.run([&](int u, int w0, int nr, const float (&acc)[32], int lane_word) {
-    // write the 32 scores of this thread's word
-    const int w = w0 + lane_word;
-    const int i0 = 32 * w;
+  core.run([&](int u, int w0, int nr, const float (&acc)[kKeysPerThread], int t) {
+    // write the 16 scores of this thread's half word
+    const int i0 = 32 * (w0 + (t >> 1)) + kKeysPerThread * (t & 1);
     if (i0 >= p.n_max) return;
     float* out = p.scores + static_cast<size_t>(u) * p.n_max;
     const float ninf = -__int_as_float(0x7f800000);
-    if (i0 + 32 <= p.n_max && (p.n_max & 3) == 0) {
+    if (i0 + kKeysPerThread <= p.n_max && (p.n_max & 3) == 0) {
 #pragma unroll
-      for (int j = 0; j < 32; j += 4) {
+      for (int j = 0; j < kKeysPerThread; j += 4) {
         float4 v;
         v.x = i0 + j + 0 < nr ? acc[j + 0] : ninf;
         v.y = i0 + j + 1 < nr ? acc[j + 1] : ninf;
@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) fathom_scan_lut_kernel(ScanPa
       }
     } else {
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
+      for (int j = 0; j < kKeysPerThread; ++j)
         if (i0 + j < p.n_max) out[i0 + j] = i0 + j < nr ? acc[j] : ninf;
     }
   });
