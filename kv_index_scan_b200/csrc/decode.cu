@@ -31,18 +31,20 @@ kvs_status fathom_scan_dispatch(const kvs_fathom_index* ix, const kvs_plan* plan
   p.n = n;
   p.n_max = n_max;
   scan_schedule(plan->B, p.G, p.b, p.nsets);
-  p.chunks_per_row = ((n_max + 31) / 32 + kChunkWords - 1) / kChunkWords;
+
   p.scores = scores;
   p.dev_status = dev_status;
   return fathom_scan_lut_launch(p, s);
 }
 
 size_t decode_ws_bytes(int R, int G, int H, int n_max, int k, int B) {
-  (void)B;
   WsCarver c(nullptr);
-  c.take<float>(static_cast<size_t>(R) * G * n_max);  // scores
-  c.take<int32_t>(static_cast<size_t>(R) * G * k);    // slots when the caller passes none
+  c.take<int32_t>(static_cast<size_t>(R) * G * k);  // slots when the caller passes none
   c.take<unsigned char>(attn_ws_bytes(R * G, H, k));
+  const size_t unfused = static_cast<size_t>(R) * G * n_max * sizeof(float);  // scores
+  const size_t fused = fused_topk_supported(n_max, k, B)
+                           ? fused_ws_bytes(R * G, n_max, k, B) : 0;
+  c.take<unsigned char>(unfused > fused ? unfused : fused);
   return c.used;
 }
 
@@ -50,26 +52,53 @@ kvs_status decode_step_run(const kvs_decode_args* a, void* ws, int32_t* dev_stat
                            cudaStream_t s) {
   const int R = a->ix->R, G = a->ix->G, RG = R * G;
   WsCarver c(ws);
-  float* scores = c.take<float>(static_cast<size_t>(RG) * a->n_max);
   int32_t* slots_ws = c.take<int32_t>(static_cast<size_t>(RG) * a->k);
   void* attn_ws = c.take<unsigned char>(attn_ws_bytes(RG, a->H, a->k));
+  void* rest = c.take<unsigned char>(0);
+  int32_t* slots = a->slots ? a->slots : slots_ws;
   kvs_status st;
   const int32_t* sel = a->idx_in;
   int shared = a->idx_in ? a->idx_shared : 0;
+  bool have_slots = false;
   if (!sel) {
+    const int B = a->plan->B;
     st = plan_bits_launch(static_cast<const float*>(a->q), a->H, a->ix->kmin, a->ix->kstep,
-                          a->ix->kvar, RG, a->plan->B, a->plan->t, a->plan->plane_idx,
-                          a->plan->plane_w, a->plan->C, s);
+                          a->ix->kvar, RG, B, a->plan->t, a->plan->plane_idx, a->plan->plane_w,
+                          a->plan->C, s);
     if (st != KVS_OK) return st;
-    st = fathom_scan_dispatch(a->ix, a->plan, a->n, a->n_max, scores, dev_status, s);
-    if (st != KVS_OK) return st;
-    st = topk_launch(scores, a->n_max, a->n, R, G, a->k, 1, a->idx, nullptr, s);
-    if (st != KVS_OK) return st;
+    if (!a->ix->host_mapped && fused_topk_supported(a->n_max, a->k, B)) {
+      // scan with on-chip top-k candidates, then the per-row merge (which also
+      // writes the slots and misses)
+      ScanParams p{};
+      p.planes = a->ix->planes;
+      p.W = a->ix->W;
+      p.RG = RG;
+      p.Gheads = G;
+      p.plane_idx = a->plan->plane_idx;
+      p.plane_w = a->plan->plane_w;
+      p.C = a->plan->C;
+      p.B = B;
+      p.n = a->n;
+      p.n_max = a->n_max;
+      scan_schedule(B, p.G, p.b, p.nsets);
+      p.dev_status = dev_status;
+      p.k = a->k;
+      st = fathom_scan_topk_launch(p, rest, a->slot_map, a->idx, slots, a->misses, s);
+      if (st != KVS_OK) return st;
+      have_slots = true;
+    } else {
+      float* scores = static_cast<float*>(rest);
+      st = fathom_scan_dispatch(a->ix, a->plan, a->n, a->n_max, scores, dev_status, s);
+      if (st != KVS_OK) return st;
+      st = topk_launch(scores, a->n_max, a->n, R, G, a->k, 1, a->idx, nullptr, s);
+      if (st != KVS_OK) return st;
+    }
     sel = a->idx;
   }
-  int32_t* slots = a->slots ? a->slots : slots_ws;
-  st = select_slots_launch(sel, shared, G, a->k, a->slot_map, a->n_max, RG, slots, a->misses, s);
-  if (st != KVS_OK) return st;
+  if (!have_slots) {
+    st = select_slots_launch(sel, shared, G, a->k, a->slot_map, a->n_max, RG, slots, a->misses, s);
+    if (st != KVS_OK) return st;
+  }
   RowSrc src{};
   src.mode = a->slot_map ? kRowsSlot : kRowsDirect;
   src.K = a->fullK;
@@ -88,13 +117,5 @@ kvs_status decode_step_run(const kvs_decode_args* a, void* ws, int32_t* dev_stat
                      attn_ws, s);
 }
 
-kvs_status lightning_scan_dispatch(const kvs_scan_args* a, float* scores, int32_t* dev_status,
-                                   cudaStream_t s) {
-  (void)a;
-  (void)scores;
-  (void)dev_status;
-  (void)s;
-  return fail(KVS_EUNSUPPORTED, "index_scan: the lightning indexer is not built yet");
-}
 
 }  // namespace kvs

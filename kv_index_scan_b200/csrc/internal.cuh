@@ -37,6 +37,10 @@ kvs_status fathom_scan_simple_launch(const uint32_t* planes, int W, int R, int G
                                      float* scores, cudaStream_t s);
 struct ScanParams;
 kvs_status fathom_scan_lut_launch(const ScanParams& p, cudaStream_t s);
+bool fused_topk_supported(int n_max, int k, int B);
+size_t fused_ws_bytes(int RG, int n_max, int k, int B);
+kvs_status fathom_scan_topk_launch(ScanParams p, void* ws, const int32_t* slot_map, int32_t* idx,
+                                   int32_t* slots, int32_t* misses, cudaStream_t s);
 kvs_status fathom_scan_dispatch(const kvs_fathom_index* ix, const kvs_plan* plan,
                                 const int32_t* n, int n_max, float* scores, int32_t* dev_status,
                                 cudaStream_t s);

@@ -1,19 +1,16 @@
 // scan_core.cuh -- the warp-specialised core of the HBM Fathom scan (see
 // scan_lut.cu for the method): TMA bulk staging of plane segments, in-register
-// 32x32 bit transposes, and bank-rotated group lookup tables. The epilogue
-// (write scores, or keep top-k candidates) is supplied by the kernel.
+// bit transposes, and bank-rotated group lookup tables. The epilogue (write
+// scores, or keep top-k candidates) is supplied by the kernel.
 #pragma once
 
 #include "internal.cuh"
 
 namespace kvs {
 
-constexpr int kScanConsumerWarps = 8;
-constexpr int kScanThreads = 32 * (kScanConsumerWarps + 1);  // + one producer warp
-constexpr int kKeysPerThread = 16;                            // half of a 32-key word
-constexpr int kChunkWords = 16 * kScanConsumerWarps;          // two consumer threads per word
-constexpr int kRowBytes = 4 * kChunkWords;                    // 512 bytes of a plane per chunk
-constexpr long long kWaitCycles = 2000000000ll;               // ~1 s bound on every wait
+constexpr int kKeysPerThread = 16;              // half of a 32-key word per consumer thread
+constexpr int kMaxScanWarps = 12;               // consumer warps per block, at most
+constexpr long long kWaitCycles = 2000000000ll;  // ~1 s bound on every wait
 
 struct ScanParams {
   const uint32_t* planes;  // [RG][D][4][W]
@@ -26,14 +23,19 @@ struct ScanParams {
   const int32_t* n;
   int n_max;
   int G, b, nsets;  // lookup schedule: G groups of b planes per set
+  int warps;        // consumer warps per block (8 or 12); a chunk is 16 * warps words
   int chunks_per_row;
   float* scores;  // unfused output [RG][n_max]
   int32_t* dev_status;
+  int nstage;  // pipeline depth (set by the launcher from the shared memory budget)
   // fused top-k candidates (scan_topk.cu)
   int k;
-  int segs_per_row;
-  uint32_t* cand_key;   // [RG][segs][k]
-  int32_t* cand_idx;    // [RG][segs][k]
+  int segs_per_row, seg_cap;
+  uint32_t* cbuf_key;   // [grid][2][cap] per-block candidate buffers: score keys
+  int32_t* cbuf_idx;    //                                             indices
+  uint64_t* cbuf_comp;  // [grid][cap] scratch for an exact cut
+  uint32_t* cand_key;   // [RG][segs][seg_cap] per-segment candidates
+  int32_t* cand_idx;
   int32_t* cand_count;  // [RG][segs]
 };
 
@@ -55,12 +57,23 @@ inline void scan_schedule(int B, int& G, int& b, int& nsets) {
   }
 }
 
-// A zero plane segment in global memory: the source of padding slots.
-__device__ __align__(16) uint32_t kZeroRow[kChunkWords];
+// Consumer warps for a schedule: 12 when two pipeline stages of 12 warps'
+// chunks still fit next to the tables (every schedule but 16 groups of 8 or 9
+// planes), else 8. More warps hide more of the scan's latency.
+__host__ __device__ constexpr int scan_warps(int G, int b) { return (G == 16 && b >= 8) ? 8 : 12; }
 
-// Dynamic shared memory of the scan kernels: [tables | stages | barriers].
-// Indexing this symbol directly keeps every table lookup a shared-memory load
-// with the base folded into the address.
+inline int scan_chunks_per_row(int n_max, int warps) {
+  const int words = (n_max + 31) / 32;
+  const int cw = 16 * warps;
+  return (words + cw - 1) / cw;
+}
+
+// A zero plane segment in global memory: the source of padding slots.
+__device__ __align__(16) uint32_t kZeroRow[16 * kMaxScanWarps];
+
+// Dynamic shared memory of the scan kernels: [tables | stages | barriers |
+// epilogue scratch]. Indexing this symbol directly keeps every table lookup a
+// shared-memory load with the base folded into the address.
 extern __shared__ __align__(1024) unsigned char g_scan_smem[];
 
 // ----------------------------------------------------------------------------- PTX helpers
@@ -106,8 +119,10 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
 }
+// Barrier of the consumer warps only (the producer warp does not take part).
+template <int W>
 __device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, %0;\n" ::"n"(32 * kScanConsumerWarps) : "memory");
+  asm volatile("bar.sync 1, %0;\n" ::"n"(32 * W) : "memory");
 }
 
 // Half of a 32x32 bit transpose, in registers. On entry x[k] holds, for one
@@ -146,21 +161,25 @@ __device__ __forceinline__ void transpose16(uint32_t (&x)[16]) {
   }
 }
 
-template <int G, int b>
+template <int G, int b, int W>
 struct ScanCore {
-  static constexpr int NPOS = G * b;            // plane slots per set
+  static constexpr int THREADS = 32 * (W + 1);   // W consumer warps + one producer warp
+  static constexpr int CHUNK_WORDS = 16 * W;     // two consumer threads per 32-key word
+  static constexpr int ROW_BYTES = 4 * CHUNK_WORDS;
+  static constexpr int NPOS = G * b;             // plane slots per set
   static constexpr int NBLK = (NPOS + 31) / 32;  // 32-plane transposes per set
   static constexpr int TBL_BYTES = (1 << b) * 128;
-  static constexpr int STAGE_BYTES = NPOS * kRowBytes;
+  static constexpr int STAGE_BYTES = NPOS * ROW_BYTES;
 
-  __host__ __device__ static int nstages(int nsets) {
-    const int budget = 220 * 1024 - nsets * TBL_BYTES - 256;
-    int s = budget / STAGE_BYTES;
+  // layout: [tables | nstage stages | 256 bytes of barriers | extra]
+  static int nstages(int nsets, size_t extra = 0) {
+    const int budget = 224 * 1024 - nsets * TBL_BYTES - 256 - static_cast<int>(extra);
+    const int s = budget / STAGE_BYTES;
     return s > 4 ? 4 : s;
   }
-  __host__ __device__ static size_t smem_bytes(int nsets) {
-    return static_cast<size_t>(nsets) * TBL_BYTES + static_cast<size_t>(nstages(nsets)) * STAGE_BYTES +
-           256;
+  static size_t smem_bytes(int nsets, size_t extra = 0) {
+    return static_cast<size_t>(nsets) * TBL_BYTES +
+           static_cast<size_t>(nstages(nsets, extra)) * STAGE_BYTES + 256 + extra;
   }
 
   const ScanParams& p;
@@ -171,11 +190,15 @@ struct ScanCore {
   int* abort_flag;
 
   __device__ explicit ScanCore(const ScanParams& params) : p(params) {
-    nstage = nstages(p.nsets);
+    nstage = p.nstage;
     stages = g_scan_smem + p.nsets * TBL_BYTES;
     full = reinterpret_cast<uint64_t*>(stages + nstage * STAGE_BYTES);
     empty = full + nstage;
     abort_flag = reinterpret_cast<int*>(empty + nstage);
+  }
+
+  __device__ unsigned char* extra() const {
+    return g_scan_smem + p.nsets * TBL_BYTES + nstage * STAGE_BYTES + 256;
   }
 
   __device__ void fail_timeout() {
@@ -203,10 +226,10 @@ struct ScanCore {
       if (*reinterpret_cast<volatile int*>(abort_flag)) break;
       int u, c, s;
       decode_item(it, u, c, s);
-      const int w0 = c * kChunkWords;
+      const int w0 = c * CHUNK_WORDS;
       const int nr = p.n[u / p.Gheads];
       const bool live = 32 * w0 < nr;
-      const int words = min(kChunkWords, p.W - w0);
+      const int words = min(CHUNK_WORDS, p.W - w0);
       const uint32_t bytes = live ? static_cast<uint32_t>(words) * 4u : 0u;
       if (lane == 0) mbar_expect_tx(&full[st], bytes * NPOS);
       __syncwarp();
@@ -218,7 +241,7 @@ struct ScanCore {
           const int slot = s * NPOS + q;
           const uint32_t* src =
               slot < p.B ? rowp + static_cast<size_t>(pidx[slot]) * p.W : kZeroRow;
-          bulk_g2s(dst0 + q * kRowBytes, src, bytes, &full[st]);
+          bulk_g2s(dst0 + q * ROW_BYTES, src, bytes, &full[st]);
         }
       }
       ++issued;
@@ -232,7 +255,7 @@ struct ScanCore {
     const int t = threadIdx.x;
     const float* w = p.plane_w + static_cast<size_t>(u) * p.B;
     const int entries = p.nsets * (1 << b) * 32;
-    for (int e = t; e < entries; e += 32 * kScanConsumerWarps) {
+    for (int e = t; e < entries; e += 32 * W) {
       const int slot = e & 31;
       const int idx = (e >> 5) & ((1 << b) - 1);
       const int s = e >> (5 + b);
@@ -249,7 +272,7 @@ struct ScanCore {
   // whose planes are rotated by lp groups.
   __device__ __forceinline__ static int slot_offset(int o, int lp) {
     const int g = o / b, bi = o % b;
-    return (((g + lp) & (G - 1)) * b + bi) * kRowBytes;
+    return (((g + lp) & (G - 1)) * b + bi) * ROW_BYTES;
   }
 
   // The set's contribution for this thread's 16 keys, added into acc. Thread
@@ -259,7 +282,13 @@ struct ScanCore {
     constexpr int NK = kKeysPerThread;
     const int t = threadIdx.x;
     const int lane = t & 31;
-    const int lp = lane % G, repl = lane / G;
+    // The two threads of a word share one rotation (so their plane loads hit
+    // the same word of a bank) and use different replicas of the tables: pair
+    // i = lane / 2 rotates by i mod G, and the 32 (rotation, replica)
+    // combinations of a warp are 32 distinct banks.
+    const int pair = lane >> 1;
+    const int lp = pair % G;
+    const int repl = (lane & 1) + 2 * (pair / G);
     const unsigned char* mine = g_scan_smem + stage_off + 4 * (t >> 1) + 2 * (t & 1);
     uint32_t prev[NK];
 #pragma unroll
@@ -304,8 +333,8 @@ struct ScanCore {
     }
   }
 
-  // Runs the pipeline over this block's items; epi(u, w0, nr, acc, t) is
-  // called by every consumer thread at the end of each chunk.
+  // Runs the pipeline over this block's chunks; epi(u, c, nr, acc, t) is
+  // called by every consumer thread at the end of each chunk c of row u.
   template <typename Epi>
   __device__ void run(Epi&& epi) {
     // whole chunks per block: the sets of a chunk accumulate in one thread
@@ -317,20 +346,21 @@ struct ScanCore {
     if (threadIdx.x == 0) {
       for (int i = 0; i < nstage; ++i) {
         mbar_init(&full[i], 1);
-        mbar_init(&empty[i], kScanConsumerWarps);
+        mbar_init(&empty[i], W);
       }
       *abort_flag = 0;
       asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     __syncthreads();
-    if (warp == kScanConsumerWarps) {
+    if (warp == W) {
       produce(beg, end);
       return;
     }
     // Consumers never leave early: after a timed-out wait they stop working
     // but keep stepping through the same items, so that every named barrier
-    // below is still met by all of them.
-    int cur_u = -1;
+    // (here and in the epilogue) is still met by all of them.
+    int cur_u = -1, row_n = 0;
+    float row_C = 0.f;
     bool dead = false;
     float acc[kKeysPerThread];
     for (int it = beg; it < end; ++it) {
@@ -338,30 +368,43 @@ struct ScanCore {
       int u, c, s;
       decode_item(it, u, c, s);
       if (u != cur_u) {
-        consumer_sync();
+        consumer_sync<W>();
         if (!dead) build_tables(u);
-        consumer_sync();
+        row_n = p.n[u / p.Gheads];
+        row_C = p.C[u];
+        consumer_sync<W>();
         cur_u = u;
       }
-      if (dead) continue;
-      if (!mbar_wait(&full[st], (k / nstage) & 1)) {
+      const int nr = row_n;
+      const int w0 = c * CHUNK_WORDS;
+      if (s == 0) {
+#pragma unroll
+        for (int j = 0; j < kKeysPerThread; ++j) acc[j] = row_C;
+      }
+      if (!dead && !mbar_wait(&full[st], (k / nstage) & 1)) {
         fail_timeout();
         dead = true;
-        continue;
       }
-      const int nr = p.n[u / p.Gheads];
-      const int w0 = c * kChunkWords;
-      if (s == 0) {
-        const float C = p.C[u];
-#pragma unroll
-        for (int j = 0; j < kKeysPerThread; ++j) acc[j] = C;
+      if (!dead) {
+        if (32 * w0 < nr) compute_set(p.nsets * TBL_BYTES + st * STAGE_BYTES, s, acc);
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[st]);
       }
-      if (32 * w0 < nr) compute_set(p.nsets * TBL_BYTES + st * STAGE_BYTES, s, acc);
-      __syncwarp();
-      if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[st]);
-      if (s == p.nsets - 1) epi(u, w0, nr, acc, static_cast<int>(threadIdx.x));
+      if (s == p.nsets - 1) epi(u, c, nr, acc, static_cast<int>(threadIdx.x));
     }
   }
 };
+
+// Calls f.template operator()<G, b, W>() for the schedule of p (G, b, warps).
+template <typename F>
+kvs_status dispatch_schedule(const ScanParams& p, F&& f) {
+#define KVS_SCHED(GG, BB) \
+  if (p.G == GG && p.b == BB) return f.template operator()<GG, BB, scan_warps(GG, BB)>();
+  KVS_SCHED(8, 1) KVS_SCHED(8, 2) KVS_SCHED(8, 3) KVS_SCHED(8, 4) KVS_SCHED(8, 5)
+  KVS_SCHED(8, 6) KVS_SCHED(8, 7) KVS_SCHED(8, 8) KVS_SCHED(8, 9)
+  KVS_SCHED(16, 5) KVS_SCHED(16, 6) KVS_SCHED(16, 7) KVS_SCHED(16, 8) KVS_SCHED(16, 9)
+#undef KVS_SCHED
+  return fail(KVS_EUNSUPPORTED, "index_scan: no lookup schedule for G=%d b=%d", p.G, p.b);
+}
 
 }  // namespace kvs

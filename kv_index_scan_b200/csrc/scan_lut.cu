@@ -25,9 +25,10 @@
 //    group g has a 2^b-entry table of the sums of its weights. One lookup per
 //    key per group replaces b multiply-adds. To keep the 32 lanes of a warp
 //    on 32 different shared-memory banks without replicating tables per lane,
-//    lane l reads its planes in an order rotated by l groups: at step g it
-//    looks up group (g + l) mod G, whose table lives in bank
-//    (g + l) mod G + G*(l div G). Tables cost 2^b * 128 bytes per set.
+//    the thread pair of lanes (2i, 2i+1) reads its planes in an order rotated
+//    by i groups: at step g it looks up group (g + i) mod G, in one of the
+//    32/G replicas of the tables, so that the 32 lanes hit 32 distinct banks.
+//    Tables cost 2^b * 128 bytes per set.
 //  * Sets. Plans with more than 144 planes are cut into sets of 16 groups of
 //    6 planes, processed one after another into the same accumulators.
 //
@@ -40,12 +41,13 @@ namespace kvs {
 
 namespace {
 
-template <int G, int b>
-__global__ void __launch_bounds__(kScanThreads, 1) fathom_scan_lut_kernel(ScanParams p) {
-  ScanCore<G, b> core(p);
-  core.run([&](int u, int w0, int nr, const float (&acc)[kKeysPerThread], int t) {
+template <int G, int b, int W>
+__global__ void __launch_bounds__(ScanCore<G, b, W>::THREADS, 1) fathom_scan_lut_kernel(ScanParams p) {
+  using Core = ScanCore<G, b, W>;
+  Core core(p);
+  core.run([&](int u, int c, int nr, const float (&acc)[kKeysPerThread], int t) {
     // write the 16 scores of this thread's half word
-    const int i0 = 32 * (w0 + (t >> 1)) + kKeysPerThread * (t & 1);
+    const int i0 = 32 * (c * Core::CHUNK_WORDS + (t >> 1)) + kKeysPerThread * (t & 1);
     if (i0 >= p.n_max) return;
     float* out = p.scores + static_cast<size_t>(u) * p.n_max;
     const float ninf = -__int_as_float(0x7f800000);
@@ -67,43 +69,31 @@ __global__ void __launch_bounds__(kScanThreads, 1) fathom_scan_lut_kernel(ScanPa
   });
 }
 
-template <int G, int b>
-kvs_status launch_gb(const ScanParams& p, cudaStream_t s) {
-  const size_t smem = ScanCore<G, b>::smem_bytes(p.nsets);
-  auto kern = fathom_scan_lut_kernel<G, b>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  const int chunks = p.RG * p.chunks_per_row;
-  if (chunks <= 0) return KVS_OK;
-  const int grid = min(chunks, sm_count());
-  kern<<<grid, kScanThreads, smem, s>>>(p);
-  return check_launch("index_scan(fathom, lut)");
-}
+struct LutLaunch {
+  const ScanParams& p;
+  cudaStream_t s;
+  template <int G, int b, int W>
+  kvs_status operator()() const {
+    using Core = ScanCore<G, b, W>;
+    const size_t smem = Core::smem_bytes(p.nsets);
+    auto kern = fathom_scan_lut_kernel<G, b, W>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    ScanParams q = p;
+    q.warps = W;
+    q.chunks_per_row = scan_chunks_per_row(p.n_max, W);
+    q.nstage = Core::nstages(p.nsets);
+    const int chunks = q.RG * q.chunks_per_row;
+    if (chunks <= 0) return KVS_OK;
+    const int grid = min(chunks, sm_count());
+    kern<<<grid, Core::THREADS, smem, s>>>(q);
+    return check_launch("index_scan(fathom, lut)");
+  }
+};
 
 }  // namespace
 
 kvs_status fathom_scan_lut_launch(const ScanParams& p, cudaStream_t s) {
-  if (p.G == 8) {
-    switch (p.b) {
-      case 1: return launch_gb<8, 1>(p, s);
-      case 2: return launch_gb<8, 2>(p, s);
-      case 3: return launch_gb<8, 3>(p, s);
-      case 4: return launch_gb<8, 4>(p, s);
-      case 5: return launch_gb<8, 5>(p, s);
-      case 6: return launch_gb<8, 6>(p, s);
-      case 7: return launch_gb<8, 7>(p, s);
-      case 8: return launch_gb<8, 8>(p, s);
-      case 9: return launch_gb<8, 9>(p, s);
-    }
-  } else {
-    switch (p.b) {
-      case 5: return launch_gb<16, 5>(p, s);
-      case 6: return launch_gb<16, 6>(p, s);
-      case 7: return launch_gb<16, 7>(p, s);
-      case 8: return launch_gb<16, 8>(p, s);
-      case 9: return launch_gb<16, 9>(p, s);
-    }
-  }
-  return fail(KVS_EUNSUPPORTED, "index_scan: no LUT schedule for G=%d b=%d", p.G, p.b);
+  return dispatch_schedule(p, LutLaunch{p, s});
 }
 
 }  // namespace kvs

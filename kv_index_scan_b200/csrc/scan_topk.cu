@@ -1,0 +1,578 @@
+// scan_topk.cu -- a2 + a3 fused for decode_step: the Fathom scan keeps each
+// row's top-k candidates on chip instead of writing every score to HBM.
+//
+// Selection order is (score desc, index asc) ("XM-Sparse: Pushing the
+// Throughput Frontier of Sparse Attention with Netpreme X-Mem", modelled
+// study: 2,048 entries are picked per layer and step).
+//
+// Scan kernel (scan_core.cuh's pipeline, this epilogue): each block walks a
+// contiguous range of chunks; the part of one (request, KV head) row inside a
+// block is a "segment". Per segment the block appends to a buffer in L2 every
+// key whose score is at least a running threshold tau (all keys, until a
+// threshold exists), as (order-preserving score key, index). When the buffer
+// may not hold another chunk, two histogram passes over the held keys (bits
+// 31..21, then 20..10) find the cell holding the k-th largest key; tau becomes
+// that cell's lower edge and every held key below it is dropped. The held set
+// always contains the segment's top-k (at least k keys are >= tau), so nothing
+// of the answer is ever lost; it is a superset, trimmed again at the segment's
+// end (and cut exactly to k only if it would still be too large).
+//
+// Merge kernel: one block per row gathers its segments' candidates as
+// distinct 53-bit composites (score key << 21 | (2^21 - 1 - index)), selects
+// exactly the k largest (five radix passes), sorts their indices ascending
+// (block radix sort), writes idx, and looks every selected key up in the
+// hot-buffer slot map (slots; misses = the number absent from the hot buffer).
+#include <cub/block/block_radix_sort.cuh>
+
+#include "internal.cuh"
+#include "scan_core.cuh"
+
+namespace kvs {
+
+namespace {
+
+constexpr int kIdxBits = 21;
+constexpr uint32_t kIdxMask = (1u << kIdxBits) - 1u;
+constexpr int kCandCap = 16384;  // per-block candidate buffer entries (two buffers)
+
+__device__ __forceinline__ uint64_t make_composite(uint32_t key, int idx) {
+  return (static_cast<uint64_t>(key) << kIdxBits) |
+         static_cast<uint64_t>(kIdxMask - static_cast<uint32_t>(idx));
+}
+__device__ __forceinline__ int composite_index(uint64_t c) {
+  return static_cast<int>(kIdxMask - static_cast<uint32_t>(c & kIdxMask));
+}
+
+// The block whose chunk range [floor(b*C/grid), floor((b+1)*C/grid)) holds chunk x.
+__host__ __device__ __forceinline__ int block_of_chunk(long long x, long long C, int grid) {
+  int b = static_cast<int>(x * grid / C);
+  while (b + 1 < grid && (static_cast<long long>(b + 1) * C) / grid <= x) ++b;
+  while (b > 0 && (static_cast<long long>(b) * C) / grid > x) --b;
+  return b;
+}
+
+// Warp 0 of a group: in a histogram over [0, nbins) bins, the bin holding
+// rank krem counted from the top; returns the bin and the count above it.
+__device__ __forceinline__ void find_bin_from_top(const unsigned* hist, int nbins, int krem,
+                                                  int& bin, int& above_out) {
+  const int lane = threadIdx.x & 31;
+  int above = 0;
+  bin = 0;
+  above_out = 0;
+  for (int top = nbins; top > 0; top -= 64) {
+    const int b0 = top - 1 - 2 * lane, b1 = b0 - 1;
+    const int c0 = b0 >= 0 ? static_cast<int>(hist[b0]) : 0;
+    const int c1 = b1 >= 0 ? static_cast<int>(hist[b1]) : 0;
+    const int mine = c0 + c1;
+    int incl = mine;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+      if (lane >= d) incl += o;
+    }
+    const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    if (above + total >= krem) {
+      const unsigned hit = __ballot_sync(0xFFFFFFFFu, above + incl >= krem);
+      const int l = __ffs(hit) - 1;
+      const int ex = __shfl_sync(0xFFFFFFFFu, incl - mine, l);
+      const int cb0 = __shfl_sync(0xFFFFFFFFu, c0, l);
+      const int bb0 = top - 1 - 2 * l;
+      if (above + ex + cb0 >= krem) {
+        bin = bb0;
+        above_out = above + ex;
+      } else {
+        bin = bb0 - 1;
+        above_out = above + ex + cb0;
+      }
+      return;
+    }
+    above += total;
+  }
+}
+
+__device__ __forceinline__ void hist_add(unsigned* hist, int bin) {
+  const int lane = threadIdx.x & 31;
+  const unsigned peers = __match_any_sync(0xFFFFFFFFu, bin);
+  if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+}
+
+struct SelectState {
+  unsigned long long prefix, mask;
+  int krem;
+  uint32_t tau;
+};
+
+// Group-wide: the kk-th largest of the n distinct 53-bit composites in src
+// (kk >= 1, n >= kk); five radix passes of 11/11/11/10/10 bits.
+template <typename Sync>
+__device__ uint64_t select_kth_composite(const uint64_t* src, int n, int kk, unsigned* hist,
+                                         SelectState* st, int tid, int nthreads, Sync sync) {
+  const int shifts[5] = {42, 31, 20, 10, 0};
+  const int widths[5] = {11, 11, 11, 10, 10};
+  if (tid == 0) {
+    st->prefix = 0ull;
+    st->mask = 0ull;
+    st->krem = kk;
+  }
+  for (int pass = 0; pass < 5; ++pass) {
+    const int shift = shifts[pass];
+    const unsigned dmask = (1u << widths[pass]) - 1u;
+    for (int b = tid; b < 2048; b += nthreads) hist[b] = 0;
+    sync();
+    const unsigned long long prefix = st->prefix, mask = st->mask;
+    for (int base = 0; base < n; base += 4 * nthreads) {
+      uint64_t c[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = base + e * nthreads + tid;
+        c[e] = i < n ? src[i] : ~0ull;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = base + e * nthreads + tid;
+        const int bin = (i < n && (c[e] & mask) == prefix) ? static_cast<int>((c[e] >> shift) & dmask) : -1;
+        hist_add(hist, bin);
+      }
+    }
+    sync();
+    if (tid < 32) {
+      int bin, above;
+      find_bin_from_top(hist, static_cast<int>(dmask) + 1, st->krem, bin, above);
+      if (tid == 0) {
+        st->prefix = prefix | (static_cast<unsigned long long>(bin) << shift);
+        st->mask = mask | (static_cast<unsigned long long>(dmask) << shift);
+        st->krem -= above;
+      }
+    }
+    sync();
+  }
+  return st->prefix;
+}
+
+struct SegState {
+  int cnt, cnt2, cur, tau_set;
+  float tau_f;
+  SelectState sel;
+};
+
+template <int G, int b, int W>
+__global__ void __launch_bounds__(ScanCore<G, b, W>::THREADS, 1) fathom_scan_topk_kernel(ScanParams p) {
+  using Core = ScanCore<G, b, W>;
+  constexpr int NT = 32 * W;
+  constexpr int CHUNK_KEYS = 32 * Core::CHUNK_WORDS;
+  Core core(p);
+  unsigned* hist = reinterpret_cast<unsigned*>(core.extra());
+  SegState* st = reinterpret_cast<SegState*>(hist + 2048);
+  auto sync = [] { consumer_sync<W>(); };
+  uint32_t* kbuf = p.cbuf_key + static_cast<size_t>(blockIdx.x) * 2 * kCandCap;
+  int32_t* ibuf = p.cbuf_idx + static_cast<size_t>(blockIdx.x) * 2 * kCandCap;
+  const long long C = static_cast<long long>(p.RG) * p.chunks_per_row;
+  if (threadIdx.x == 0) {
+    st->cnt = 0;
+    st->cur = 0;
+    st->tau_set = 0;
+  }
+  // (visible to the consumers through the barrier at the first row change)
+
+  // Lower edge of the 22-bit key cell holding the kk-th largest held key
+  // (two histogram passes; at least kk held keys are >= it).
+  auto cell_threshold = [&](const uint32_t* keys, int n, int kk) -> uint32_t {
+    const int t = threadIdx.x;
+    for (int bb = t; bb < 2048; bb += NT) hist[bb] = 0;
+    sync();
+    for (int base = 0; base < n; base += 4 * NT) {
+      uint32_t kv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = base + e * NT + t;
+        kv[e] = i < n ? keys[i] : 0u;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        hist_add(hist, base + e * NT + t < n ? static_cast<int>(kv[e] >> 21) : -1);
+    }
+    sync();
+    if (t < 32) {
+      int bin, above;
+      find_bin_from_top(hist, 2048, kk, bin, above);
+      if (t == 0) {
+        st->sel.tau = static_cast<uint32_t>(bin);
+        st->sel.krem = kk - above;
+      }
+    }
+    sync();
+    const uint32_t b1 = st->sel.tau;
+    for (int bb = t; bb < 2048; bb += NT) hist[bb] = 0;
+    sync();
+    for (int base = 0; base < n; base += 4 * NT) {
+      uint32_t kv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = base + e * NT + t;
+        kv[e] = i < n ? keys[i] : 0u;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool in = base + e * NT + t < n && (kv[e] >> 21) == b1;
+        hist_add(hist, in ? static_cast<int>((kv[e] >> 10) & 2047u) : -1);
+      }
+    }
+    sync();
+    if (t < 32) {
+      int bin, above;
+      find_bin_from_top(hist, 2048, st->sel.krem, bin, above);
+      if (t == 0) st->sel.tau = (b1 << 21) | (static_cast<uint32_t>(bin) << 10);
+    }
+    sync();
+    return st->sel.tau;
+  };
+
+  // Keep the held keys >= tau, moved into the other buffer (uniform call).
+  auto keep_at_least = [&](uint32_t tau) {
+    const int t = threadIdx.x;
+    const int n = st->cnt;
+    const uint32_t* ks = kbuf + static_cast<size_t>(st->cur) * kCandCap;
+    const int32_t* is = ibuf + static_cast<size_t>(st->cur) * kCandCap;
+    uint32_t* kd = kbuf + static_cast<size_t>(st->cur ^ 1) * kCandCap;
+    int32_t* id = ibuf + static_cast<size_t>(st->cur ^ 1) * kCandCap;
+    if (t == 0) st->cnt2 = 0;
+    sync();
+    for (int base = 0; base < n; base += NT) {
+      const int i = base + t;
+      const uint32_t key = i < n ? ks[i] : 0u;
+      const bool take = i < n && key >= tau;
+      const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
+      if (m == 0u) continue;
+      const int lane = t & 31, leader = __ffs(m) - 1;
+      int pos = 0;
+      if (lane == leader) pos = atomicAdd(&st->cnt2, __popc(m));
+      pos = __shfl_sync(0xFFFFFFFFu, pos, leader) + __popc(m & ((1u << lane) - 1u));
+      if (take) {
+        kd[pos] = key;
+        id[pos] = is[i];
+      }
+    }
+    sync();
+    if (t == 0) {
+      st->cnt = st->cnt2;
+      st->cur ^= 1;
+      st->tau_set = 1;
+      st->tau_f = key_to_float(tau);
+    }
+    sync();
+  };
+
+  // Exact cut to the best kk held keys; only when a cell holds so many equal
+  // keys that the cell threshold cannot shrink the set (uniform call).
+  auto cut_exact = [&](int kk) {
+    const int t = threadIdx.x;
+    const int n = st->cnt;
+    const uint32_t* ks = kbuf + static_cast<size_t>(st->cur) * kCandCap;
+    const int32_t* is = ibuf + static_cast<size_t>(st->cur) * kCandCap;
+    uint64_t* comp = p.cbuf_comp + static_cast<size_t>(blockIdx.x) * kCandCap;
+    for (int i = t; i < n; i += NT) comp[i] = make_composite(ks[i], is[i]);
+    sync();
+    const uint64_t tau = select_kth_composite(comp, n, min(kk, n), hist, &st->sel, t, NT, sync);
+    uint32_t* kd = reinterpret_cast<uint32_t*>(ibuf + static_cast<size_t>(st->cur ^ 1) * kCandCap);
+    if (t == 0) st->cnt2 = 0;
+    sync();
+    // kept entries as (key, index) pairs in the other buffer's index array,
+    // then copied back over the current buffer
+    for (int base = 0; base < n; base += NT) {
+      const int i = base + t;
+      const uint64_t c = i < n ? comp[i] : 0ull;
+      const bool take = i < n && c >= tau;
+      const unsigned msk = __ballot_sync(0xFFFFFFFFu, take);
+      if (msk == 0u) continue;
+      const int lane = t & 31, leader = __ffs(msk) - 1;
+      int pos = 0;
+      if (lane == leader) pos = atomicAdd(&st->cnt2, __popc(msk));
+      pos = __shfl_sync(0xFFFFFFFFu, pos, leader) + __popc(msk & ((1u << lane) - 1u));
+      if (take) {
+        kd[2 * pos] = static_cast<uint32_t>(c >> kIdxBits);
+        kd[2 * pos + 1] = static_cast<uint32_t>(composite_index(c));
+      }
+    }
+    sync();
+    uint32_t* kc = kbuf + static_cast<size_t>(st->cur) * kCandCap;
+    int32_t* ic = ibuf + static_cast<size_t>(st->cur) * kCandCap;
+    const int kept = st->cnt2;
+    for (int i = t; i < kept; i += NT) {
+      kc[i] = kd[2 * i];
+      ic[i] = static_cast<int32_t>(kd[2 * i + 1]);
+    }
+    sync();
+    if (t == 0) {
+      st->cnt = kept;
+      st->tau_set = 1;
+      st->tau_f = key_to_float(static_cast<uint32_t>(tau >> kIdxBits));
+    }
+    sync();
+  };
+
+  // Trim the held set to a superset of its top kk (uniform call).
+  auto trim = [&](int kk) {
+    if (st->cnt <= kk) return;
+    const uint32_t tau = cell_threshold(kbuf + static_cast<size_t>(st->cur) * kCandCap, st->cnt, kk);
+    keep_at_least(tau);
+  };
+
+  core.run([&](int u, int c, int nr, const float (&acc)[kKeysPerThread], int t) {
+    // 1. keys at or above the running threshold join the segment's candidates
+    const int i0 = 32 * (c * Core::CHUNK_WORDS + (t >> 1)) + kKeysPerThread * (t & 1);
+    const bool has_tau = st->tau_set != 0;
+    const float tau = st->tau_f;
+    uint32_t* kb = kbuf + static_cast<size_t>(st->cur) * kCandCap;
+    int32_t* ib = ibuf + static_cast<size_t>(st->cur) * kCandCap;
+#pragma unroll
+    for (int j = 0; j < kKeysPerThread; ++j) {
+      const int i = i0 + j;
+      const bool take = i < nr && (!has_tau || acc[j] >= tau);
+      const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
+      if (m == 0u) continue;
+      const int lane = threadIdx.x & 31;
+      const int leader = __ffs(m) - 1;
+      int base = 0;
+      if (lane == leader) base = atomicAdd(&st->cnt, __popc(m));
+      base = __shfl_sync(0xFFFFFFFFu, base, leader) + __popc(m & ((1u << lane) - 1u));
+      if (take) {
+        kb[base] = ordered_key(acc[j]);
+        ib[base] = i;
+      }
+    }
+    sync();
+    // 2. the segment ends here, or there must be room for one more chunk
+    const long long chunk_id = static_cast<long long>(u) * p.chunks_per_row + c;
+    const long long last_chunk = static_cast<long long>(blockIdx.x + 1) * C / gridDim.x - 1;
+    const bool seg_end = c == p.chunks_per_row - 1 || chunk_id == last_chunk;
+    if (seg_end) {
+      trim(p.k);
+      if (st->cnt > p.seg_cap) cut_exact(p.k);
+      const int kk = st->cnt;
+      const int slot = static_cast<int>(blockIdx.x) -
+                       block_of_chunk(static_cast<long long>(u) * p.chunks_per_row, C, gridDim.x);
+      const size_t off = (static_cast<size_t>(u) * p.segs_per_row + slot) * p.seg_cap;
+      const uint32_t* ks = kbuf + static_cast<size_t>(st->cur) * kCandCap;
+      const int32_t* is = ibuf + static_cast<size_t>(st->cur) * kCandCap;
+      for (int e = threadIdx.x; e < kk; e += NT) {
+        p.cand_key[off + e] = ks[e];
+        p.cand_idx[off + e] = is[e];
+      }
+      if (threadIdx.x == 0) {
+        p.cand_count[static_cast<size_t>(u) * p.segs_per_row + slot] = kk;
+        st->cnt = 0;
+        st->tau_set = 0;
+      }
+      sync();
+    } else if (st->cnt > kCandCap - CHUNK_KEYS) {
+      trim(p.k);
+      if (st->cnt > kCandCap - CHUNK_KEYS) cut_exact(p.k);
+    }
+  });
+}
+
+// One block per (r, g): gather the segments' candidates, select, sort, slot
+// lookup. 1024 threads, up to 4096 selected.
+constexpr int kMergeThreads = 1024;
+constexpr int kMergeItems = 4;
+constexpr int kMergeSmemEntries = 20480;
+
+__global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(
+    ScanParams p, int scan_grid, uint64_t* __restrict__ gscratch,
+    const int32_t* __restrict__ slot_map, int32_t* __restrict__ idx, int32_t* __restrict__ slots,
+    int32_t* __restrict__ misses) {
+  using Sort = cub::BlockRadixSort<uint32_t, kMergeThreads, kMergeItems>;
+  // the select's histogram, the chosen indices and the sort's scratch are
+  // used one after another, separated by barriers: one union
+  __shared__ union {
+    unsigned hist[2048];
+    uint32_t chosen[kMergeThreads * kMergeItems];
+    typename Sort::TempStorage sort;
+  } sm;
+  __shared__ SelectState sel;
+  __shared__ int seg_count[64], seg_off[65];
+  __shared__ int nsel;
+  __shared__ int miss_warp[kMergeThreads / 32];
+  extern __shared__ __align__(16) uint64_t comp_smem[];
+  const int u = blockIdx.x;
+  const int t = threadIdx.x;
+  const int nr = p.n[u / p.Gheads];
+  const int kk = min(p.k, nr);
+  const long long C = static_cast<long long>(p.RG) * p.chunks_per_row;
+  const int b0 = block_of_chunk(static_cast<long long>(u) * p.chunks_per_row, C, scan_grid);
+  const int b1 = block_of_chunk(static_cast<long long>(u + 1) * p.chunks_per_row - 1, C, scan_grid);
+  const int segs = b1 - b0 + 1;
+  if (t < segs) seg_count[t] = p.cand_count[static_cast<size_t>(u) * p.segs_per_row + t];
+  __syncthreads();
+  if (t == 0) {
+    int o = 0;
+    for (int s = 0; s < segs; ++s) {
+      seg_off[s] = o;
+      o += seg_count[s];
+    }
+    seg_off[segs] = o;
+    nsel = 0;
+  }
+  __syncthreads();
+  const int total = seg_off[segs];
+  uint64_t* comp = total <= kMergeSmemEntries
+                       ? comp_smem
+                       : gscratch + static_cast<size_t>(u) * p.segs_per_row * p.seg_cap;
+  for (int s = 0; s < segs; ++s) {
+    const size_t off = (static_cast<size_t>(u) * p.segs_per_row + s) * p.seg_cap;
+    for (int i = t; i < seg_count[s]; i += kMergeThreads)
+      comp[seg_off[s] + i] = make_composite(p.cand_key[off + i], p.cand_idx[off + i]);
+  }
+  __syncthreads();
+  uint64_t tau = 0ull;
+  if (kk > 0 && total > kk)
+    tau = select_kth_composite(comp, total, kk, sm.hist, &sel, t, kMergeThreads,
+                               [] { __syncthreads(); });
+  __syncthreads();
+  // the selected indices, unordered, into the blocked sort input
+  uint32_t* chosen = sm.chosen;
+  for (int base = 0; base < total; base += kMergeThreads) {
+    const int i = base + t;
+    const uint64_t c = i < total ? comp[i] : 0ull;
+    const bool take = kk > 0 && i < total && c >= tau;
+    const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
+    if (m) {
+      const int lane = t & 31, leader = __ffs(m) - 1;
+      int basew = 0;
+      if (lane == leader) basew = atomicAdd(&nsel, __popc(m));
+      basew = __shfl_sync(0xFFFFFFFFu, basew, leader);
+      const int pos = basew + __popc(m & ((1u << lane) - 1u));
+      if (take && pos < kMergeThreads * kMergeItems) chosen[pos] = composite_index(c);
+    }
+  }
+  __syncthreads();
+  const int nchosen = min(nsel, kk);
+  uint32_t keys[kMergeItems];
+#pragma unroll
+  for (int e = 0; e < kMergeItems; ++e) {
+    const int i = t * kMergeItems + e;
+    keys[e] = i < nchosen ? chosen[i] : 0xFFFFFFFFu;
+  }
+  __syncthreads();
+  Sort(sm.sort).Sort(keys);
+  int my_miss = 0;
+#pragma unroll
+  for (int e = 0; e < kMergeItems; ++e) {
+    const int j = t * kMergeItems + e;
+    if (j >= p.k) continue;
+    const int i = j < nchosen ? static_cast<int>(keys[e]) : -1;
+    idx[static_cast<size_t>(u) * p.k + j] = i;
+    int s = -2;
+    if (i >= 0) {
+      s = slot_map ? slot_map[static_cast<size_t>(u) * p.n_max + i] : -1;
+      my_miss += s < 0 ? 1 : 0;
+    }
+    if (slots) slots[static_cast<size_t>(u) * p.k + j] = s;
+  }
+  const int w = __reduce_add_sync(0xFFFFFFFFu, my_miss);
+  if ((t & 31) == 0) miss_warp[t >> 5] = w;
+  __syncthreads();
+  if (t == 0 && misses) {
+    int m = 0;
+    for (int e = 0; e < kMergeThreads / 32; ++e) m += miss_warp[e];
+    misses[u] = m;
+  }
+}
+
+int fused_grid(int RG, int cpr) {
+  const long long C = static_cast<long long>(RG) * cpr;
+  return static_cast<int>(C < sm_count() ? C : sm_count());
+}
+
+int fused_segs_per_row(int RG, int cpr, int grid) {
+  const long long C = static_cast<long long>(RG) * cpr;
+  int mx = 1;
+  for (int u = 0; u < RG; ++u) {
+    const int b0 = block_of_chunk(static_cast<long long>(u) * cpr, C, grid);
+    const int b1 = block_of_chunk(static_cast<long long>(u + 1) * cpr - 1, C, grid);
+    mx = max(mx, b1 - b0 + 1);
+  }
+  return mx;
+}
+
+struct Layout {
+  int grid, cpr, segs, seg_cap;
+};
+
+Layout fused_layout(int RG, int n_max, int k, int B) {
+  int G, b, nsets;
+  scan_schedule(B, G, b, nsets);
+  Layout L{};
+  L.cpr = scan_chunks_per_row(n_max, scan_warps(G, b));
+  L.grid = fused_grid(RG, L.cpr);
+  L.segs = L.grid > 0 ? fused_segs_per_row(RG, L.cpr, L.grid) : 1;
+  L.seg_cap = 2 * k;
+  return L;
+}
+
+struct FusedLaunch {
+  const ScanParams& p;
+  int grid;
+  cudaStream_t s;
+  template <int G, int b, int W>
+  kvs_status operator()() const {
+    using Core = ScanCore<G, b, W>;
+    const size_t extra = 2048 * sizeof(unsigned) + sizeof(SegState);
+    const size_t smem = Core::smem_bytes(p.nsets, extra);
+    auto kern = fathom_scan_topk_kernel<G, b, W>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    ScanParams q = p;
+    q.warps = W;
+    q.nstage = Core::nstages(p.nsets, extra);
+    kern<<<grid, Core::THREADS, smem, s>>>(q);
+    return check_launch("decode_step(scan+topk)");
+  }
+};
+
+}  // namespace
+
+bool fused_topk_supported(int n_max, int k, int B) {
+  return B > 0 && k >= 1 && k <= kMergeThreads * kMergeItems && 2 * k <= kCandCap - 6144 &&
+         n_max <= (1 << kIdxBits);
+}
+
+size_t fused_ws_bytes(int RG, int n_max, int k, int B) {
+  const Layout L = fused_layout(RG, n_max, k, B);
+  WsCarver c(nullptr);
+  c.take<uint32_t>(static_cast<size_t>(L.grid) * 2 * kCandCap);
+  c.take<int32_t>(static_cast<size_t>(L.grid) * 2 * kCandCap);
+  c.take<uint64_t>(static_cast<size_t>(L.grid) * kCandCap);
+  c.take<uint32_t>(static_cast<size_t>(RG) * L.segs * L.seg_cap);
+  c.take<int32_t>(static_cast<size_t>(RG) * L.segs * L.seg_cap);
+  c.take<int32_t>(static_cast<size_t>(RG) * L.segs);
+  c.take<uint64_t>(static_cast<size_t>(RG) * L.segs * L.seg_cap);
+  return c.used;
+}
+
+kvs_status fathom_scan_topk_launch(ScanParams p, void* ws, const int32_t* slot_map, int32_t* idx,
+                                   int32_t* slots, int32_t* misses, cudaStream_t s) {
+  const Layout L = fused_layout(p.RG, p.n_max, p.k, p.B);
+  if (L.grid <= 0) return KVS_OK;
+  if (L.segs > 64) return fail(KVS_EUNSUPPORTED, "decode_step: %d segments per row", L.segs);
+  p.chunks_per_row = L.cpr;
+  p.segs_per_row = L.segs;
+  p.seg_cap = L.seg_cap;
+  WsCarver c(ws);
+  p.cbuf_key = c.take<uint32_t>(static_cast<size_t>(L.grid) * 2 * kCandCap);
+  p.cbuf_idx = c.take<int32_t>(static_cast<size_t>(L.grid) * 2 * kCandCap);
+  p.cbuf_comp = c.take<uint64_t>(static_cast<size_t>(L.grid) * kCandCap);
+  p.cand_key = c.take<uint32_t>(static_cast<size_t>(p.RG) * L.segs * L.seg_cap);
+  p.cand_idx = c.take<int32_t>(static_cast<size_t>(p.RG) * L.segs * L.seg_cap);
+  p.cand_count = c.take<int32_t>(static_cast<size_t>(p.RG) * L.segs);
+  uint64_t* gscratch = c.take<uint64_t>(static_cast<size_t>(p.RG) * L.segs * L.seg_cap);
+  kvs_status st = dispatch_schedule(p, FusedLaunch{p, L.grid, s});
+  if (st != KVS_OK) return st;
+  const size_t msmem = static_cast<size_t>(kMergeSmemEntries) * sizeof(uint64_t);
+  cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       static_cast<int>(msmem));
+  topk_merge_kernel<<<p.RG, kMergeThreads, msmem, s>>>(p, L.grid, gscratch, slot_map, idx, slots,
+                                                        misses);
+  return check_launch("decode_step(top-k merge)");
+}
+
+}  // namespace kvs

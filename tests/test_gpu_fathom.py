@@ -259,3 +259,18 @@ def test_decode_step_layer_sharing_reuses_selection(kvs):
     torch.cuda.synchronize()
     assert torch.all(step.idx == -7)  # not written when a selection is given
     assert torch.equal(step.out, out1)
+
+
+def test_decode_step_all_scores_tied_takes_first_indices(kvs):
+    """Degenerate keys: every key of a row equal -> zero quantiser step, all
+    codes 0, every score equal -> the top-k is the first k indices."""
+    R, G, H, n, k, S = 2, 2, 4, 9000, 2048, 4096
+    K = torch.full((R, G, n, D), 0.5, dtype=torch.bfloat16)
+    V = synth.fathom_kv(R, G, D, n, seed=31)[1]
+    q = synth.queries(R, G, H, D, seed=31)
+    ix = kvs.build_fathom_index(K.to(DEV), [n, n])
+    step = kvs.DecodeStep(ix, [n, n], n, H, 92, k, K.to(DEV), V.to(DEV))
+    step(q.to(DEV))
+    torch.cuda.synchronize()
+    assert torch.equal(step.idx.cpu(), torch.arange(k, dtype=torch.int32).expand(R, G, k))
+    assert torch.all(step.misses == k)
