@@ -228,7 +228,7 @@ def run_ours(args, cfg, dist, rank, ws):
     plan = step.plan
 
     def scan_once():
-        kvs.index_scan_fathom(data["index"], plan, data["nl"], cfg["n"], scores=scan_scores)
+        kvs.index_scan_fathom(data["index"], plan, step.n, cfg["n"], scores=scan_scores)
 
     scan_ms = time_steps(scan_once, max(args.steps, 5), 3, stream)
 

@@ -31,6 +31,7 @@ struct ScanParams {
   // fused top-k candidates (scan_topk.cu)
   int k;
   int segs_per_row, seg_cap;
+  int cand_cap, trim_at;  // per-block candidate capacity, and the count that triggers a trim
   uint32_t* cbuf_key;   // [grid][2][cap] per-block candidate buffers: score keys
   int32_t* cbuf_idx;    //                                             indices
   uint64_t* cbuf_comp;  // [grid][cap] scratch for an exact cut
@@ -67,6 +68,14 @@ inline int scan_chunks_per_row(int n_max, int warps) {
   const int cw = 16 * warps;
   return (words + cw - 1) / cw;
 }
+
+// Register budget of the scan kernels: one block per SM. 128 registers a
+// thread hold every schedule without spills and timed no slower than the
+// whole file the block size leaves (B = 92 and 136 at 128K keys a row).
+#ifndef KVS_SCAN_MAXNREG
+#define KVS_SCAN_MAXNREG 128
+#endif
+#define KVS_SCAN_BOUNDS(G, b, W) __maxnreg__(KVS_SCAN_MAXNREG)
 
 // A zero plane segment in global memory: the source of padding slots.
 __device__ __align__(16) uint32_t kZeroRow[16 * kMaxScanWarps];

@@ -42,7 +42,7 @@ namespace kvs {
 namespace {
 
 template <int G, int b, int W>
-__global__ void __launch_bounds__(ScanCore<G, b, W>::THREADS, 1) fathom_scan_lut_kernel(ScanParams p) {
+__global__ void KVS_SCAN_BOUNDS(G, b, W) fathom_scan_lut_kernel(ScanParams p) {
   using Core = ScanCore<G, b, W>;
   Core core(p);
   core.run([&](int u, int c, int nr, const float (&acc)[kKeysPerThread], int t) {

@@ -33,7 +33,7 @@ namespace {
 
 constexpr int kIdxBits = 21;
 constexpr uint32_t kIdxMask = (1u << kIdxBits) - 1u;
-constexpr int kCandCap = 16384;  // per-block candidate buffer entries (two buffers)
+constexpr int kCandCap = 16384;  // per-block candidate buffer entries in global memory
 
 __device__ __forceinline__ uint64_t make_composite(uint32_t key, int idx) {
   return (static_cast<uint64_t>(key) << kIdxBits) |
@@ -150,33 +150,34 @@ __device__ uint64_t select_kth_composite(const uint64_t* src, int n, int kk, uns
 }
 
 struct SegState {
-  int cnt, cnt2, cur, tau_set;
+  int cnt, cnt2, tau_set;
   float tau_f;
   SelectState sel;
 };
 
-template <int G, int b, int W>
-__global__ void __launch_bounds__(ScanCore<G, b, W>::THREADS, 1) fathom_scan_topk_kernel(ScanParams p) {
+// Candidate store of one block: keys in shared memory (SK) or in global
+// memory, indices in global memory; one buffer, compacted in place.
+template <int G, int b, int W, bool SK>
+__global__ void KVS_SCAN_BOUNDS(G, b, W) fathom_scan_topk_kernel(ScanParams p) {
   using Core = ScanCore<G, b, W>;
   constexpr int NT = 32 * W;
-  constexpr int CHUNK_KEYS = 32 * Core::CHUNK_WORDS;
   Core core(p);
   unsigned* hist = reinterpret_cast<unsigned*>(core.extra());
   SegState* st = reinterpret_cast<SegState*>(hist + 2048);
   auto sync = [] { consumer_sync<W>(); };
-  uint32_t* kbuf = p.cbuf_key + static_cast<size_t>(blockIdx.x) * 2 * kCandCap;
-  int32_t* ibuf = p.cbuf_idx + static_cast<size_t>(blockIdx.x) * 2 * kCandCap;
+  uint32_t* kb = SK ? reinterpret_cast<uint32_t*>(st + 1)
+                    : p.cbuf_key + static_cast<size_t>(blockIdx.x) * p.cand_cap;
+  int32_t* ib = p.cbuf_idx + static_cast<size_t>(blockIdx.x) * p.cand_cap;
   const long long C = static_cast<long long>(p.RG) * p.chunks_per_row;
   if (threadIdx.x == 0) {
     st->cnt = 0;
-    st->cur = 0;
     st->tau_set = 0;
   }
   // (visible to the consumers through the barrier at the first row change)
 
   // Lower edge of the 22-bit key cell holding the kk-th largest held key
   // (two histogram passes; at least kk held keys are >= it).
-  auto cell_threshold = [&](const uint32_t* keys, int n, int kk) -> uint32_t {
+  auto cell_threshold = [&](int n, int kk) -> uint32_t {
     const int t = threadIdx.x;
     for (int bb = t; bb < 2048; bb += NT) hist[bb] = 0;
     sync();
@@ -185,7 +186,7 @@ __global__ void __launch_bounds__(ScanCore<G, b, W>::THREADS, 1) fathom_scan_top
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int i = base + e * NT + t;
-        kv[e] = i < n ? keys[i] : 0u;
+        kv[e] = i < n ? kb[i] : 0u;
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e)
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(ScanCore<G, b, W>::THREADS, 1) fathom_scan_top
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int i = base + e * NT + t;
-        kv[e] = i < n ? keys[i] : 0u;
+        kv[e] = i < n ? kb[i] : 0u;
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -227,20 +228,61 @@ __global__ void __launch_bounds__(ScanCore<G, b, W>::THREADS, 1) fathom_scan_top
     return st->sel.tau;
   };
 
-  // Keep the held keys >= tau, moved into the other buffer (uniform call).
-  auto keep_at_least = [&](uint32_t tau) {
+  // Keep the held entries with key >= tau, compacted in place: each round
+  // reads one entry per thread, then (after a barrier) writes the kept ones
+  // below it, so no unread entry is ever overwritten (uniform call).
+  auto keep_at_least = [&](uint32_t tau, float tau_f) {
     const int t = threadIdx.x;
     const int n = st->cnt;
-    const uint32_t* ks = kbuf + static_cast<size_t>(st->cur) * kCandCap;
-    const int32_t* is = ibuf + static_cast<size_t>(st->cur) * kCandCap;
-    uint32_t* kd = kbuf + static_cast<size_t>(st->cur ^ 1) * kCandCap;
-    int32_t* id = ibuf + static_cast<size_t>(st->cur ^ 1) * kCandCap;
     if (t == 0) st->cnt2 = 0;
     sync();
     for (int base = 0; base < n; base += NT) {
       const int i = base + t;
-      const uint32_t key = i < n ? ks[i] : 0u;
+      uint32_t key = 0u;
+      int32_t ix = 0;
+      if (i < n) {
+        key = kb[i];
+        ix = ib[i];
+      }
       const bool take = i < n && key >= tau;
+      sync();
+      const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
+      if (m) {
+        const int lane = t & 31, leader = __ffs(m) - 1;
+        int pos = 0;
+        if (lane == leader) pos = atomicAdd(&st->cnt2, __popc(m));
+        pos = __shfl_sync(0xFFFFFFFFu, pos, leader) + __popc(m & ((1u << lane) - 1u));
+        if (take) {
+          kb[pos] = key;
+          ib[pos] = ix;
+        }
+      }
+    }
+    sync();
+    if (t == 0) {
+      st->cnt = st->cnt2;
+      st->tau_set = 1;
+      st->tau_f = tau_f;
+    }
+    sync();
+  };
+
+  // Exact cut to the best kk held entries by (key, index) composites; only
+  // when a cell holds so many equal keys that the cell threshold cannot
+  // shrink the set (uniform call).
+  auto cut_exact = [&](int kk) {
+    const int t = threadIdx.x;
+    const int n = st->cnt;
+    uint64_t* comp = p.cbuf_comp + static_cast<size_t>(blockIdx.x) * p.cand_cap;
+    for (int i = t; i < n; i += NT) comp[i] = make_composite(kb[i], ib[i]);
+    sync();
+    const uint64_t tau = select_kth_composite(comp, n, min(kk, n), hist, &st->sel, t, NT, sync);
+    if (t == 0) st->cnt2 = 0;
+    sync();
+    for (int base = 0; base < n; base += NT) {
+      const int i = base + t;
+      const uint64_t c = i < n ? comp[i] : 0ull;
+      const bool take = i < n && c >= tau;
       const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
       if (m == 0u) continue;
       const int lane = t & 31, leader = __ffs(m) - 1;
@@ -248,62 +290,13 @@ __global__ void __launch_bounds__(ScanCore<G, b, W>::THREADS, 1) fathom_scan_top
       if (lane == leader) pos = atomicAdd(&st->cnt2, __popc(m));
       pos = __shfl_sync(0xFFFFFFFFu, pos, leader) + __popc(m & ((1u << lane) - 1u));
       if (take) {
-        kd[pos] = key;
-        id[pos] = is[i];
+        kb[pos] = static_cast<uint32_t>(c >> kIdxBits);
+        ib[pos] = composite_index(c);
       }
     }
     sync();
     if (t == 0) {
       st->cnt = st->cnt2;
-      st->cur ^= 1;
-      st->tau_set = 1;
-      st->tau_f = key_to_float(tau);
-    }
-    sync();
-  };
-
-  // Exact cut to the best kk held keys; only when a cell holds so many equal
-  // keys that the cell threshold cannot shrink the set (uniform call).
-  auto cut_exact = [&](int kk) {
-    const int t = threadIdx.x;
-    const int n = st->cnt;
-    const uint32_t* ks = kbuf + static_cast<size_t>(st->cur) * kCandCap;
-    const int32_t* is = ibuf + static_cast<size_t>(st->cur) * kCandCap;
-    uint64_t* comp = p.cbuf_comp + static_cast<size_t>(blockIdx.x) * kCandCap;
-    for (int i = t; i < n; i += NT) comp[i] = make_composite(ks[i], is[i]);
-    sync();
-    const uint64_t tau = select_kth_composite(comp, n, min(kk, n), hist, &st->sel, t, NT, sync);
-    uint32_t* kd = reinterpret_cast<uint32_t*>(ibuf + static_cast<size_t>(st->cur ^ 1) * kCandCap);
-    if (t == 0) st->cnt2 = 0;
-    sync();
-    // kept entries as (key, index) pairs in the other buffer's index array,
-    // then copied back over the current buffer
-    for (int base = 0; base < n; base += NT) {
-      const int i = base + t;
-      const uint64_t c = i < n ? comp[i] : 0ull;
-      const bool take = i < n && c >= tau;
-      const unsigned msk = __ballot_sync(0xFFFFFFFFu, take);
-      if (msk == 0u) continue;
-      const int lane = t & 31, leader = __ffs(msk) - 1;
-      int pos = 0;
-      if (lane == leader) pos = atomicAdd(&st->cnt2, __popc(msk));
-      pos = __shfl_sync(0xFFFFFFFFu, pos, leader) + __popc(msk & ((1u << lane) - 1u));
-      if (take) {
-        kd[2 * pos] = static_cast<uint32_t>(c >> kIdxBits);
-        kd[2 * pos + 1] = static_cast<uint32_t>(composite_index(c));
-      }
-    }
-    sync();
-    uint32_t* kc = kbuf + static_cast<size_t>(st->cur) * kCandCap;
-    int32_t* ic = ibuf + static_cast<size_t>(st->cur) * kCandCap;
-    const int kept = st->cnt2;
-    for (int i = t; i < kept; i += NT) {
-      kc[i] = kd[2 * i];
-      ic[i] = static_cast<int32_t>(kd[2 * i + 1]);
-    }
-    sync();
-    if (t == 0) {
-      st->cnt = kept;
       st->tau_set = 1;
       st->tau_f = key_to_float(static_cast<uint32_t>(tau >> kIdxBits));
     }
@@ -313,8 +306,8 @@ __global__ void __launch_bounds__(ScanCore<G, b, W>::THREADS, 1) fathom_scan_top
   // Trim the held set to a superset of its top kk (uniform call).
   auto trim = [&](int kk) {
     if (st->cnt <= kk) return;
-    const uint32_t tau = cell_threshold(kbuf + static_cast<size_t>(st->cur) * kCandCap, st->cnt, kk);
-    keep_at_least(tau);
+    const uint32_t tau = cell_threshold(st->cnt, kk);
+    keep_at_least(tau, key_to_float(tau));
   };
 
   core.run([&](int u, int c, int nr, const float (&acc)[kKeysPerThread], int t) {
@@ -322,8 +315,6 @@ __global__ void __launch_bounds__(ScanCore<G, b, W>::THREADS, 1) fathom_scan_top
     const int i0 = 32 * (c * Core::CHUNK_WORDS + (t >> 1)) + kKeysPerThread * (t & 1);
     const bool has_tau = st->tau_set != 0;
     const float tau = st->tau_f;
-    uint32_t* kb = kbuf + static_cast<size_t>(st->cur) * kCandCap;
-    int32_t* ib = ibuf + static_cast<size_t>(st->cur) * kCandCap;
 #pragma unroll
     for (int j = 0; j < kKeysPerThread; ++j) {
       const int i = i0 + j;
@@ -352,11 +343,9 @@ __global__ void __launch_bounds__(ScanCore<G, b, W>::THREADS, 1) fathom_scan_top
       const int slot = static_cast<int>(blockIdx.x) -
                        block_of_chunk(static_cast<long long>(u) * p.chunks_per_row, C, gridDim.x);
       const size_t off = (static_cast<size_t>(u) * p.segs_per_row + slot) * p.seg_cap;
-      const uint32_t* ks = kbuf + static_cast<size_t>(st->cur) * kCandCap;
-      const int32_t* is = ibuf + static_cast<size_t>(st->cur) * kCandCap;
       for (int e = threadIdx.x; e < kk; e += NT) {
-        p.cand_key[off + e] = ks[e];
-        p.cand_idx[off + e] = is[e];
+        p.cand_key[off + e] = kb[e];
+        p.cand_idx[off + e] = ib[e];
       }
       if (threadIdx.x == 0) {
         p.cand_count[static_cast<size_t>(u) * p.segs_per_row + slot] = kk;
@@ -364,9 +353,9 @@ __global__ void __launch_bounds__(ScanCore<G, b, W>::THREADS, 1) fathom_scan_top
         st->tau_set = 0;
       }
       sync();
-    } else if (st->cnt > kCandCap - CHUNK_KEYS) {
+    } else if (st->cnt > p.trim_at) {
       trim(p.k);
-      if (st->cnt > kCandCap - CHUNK_KEYS) cut_exact(p.k);
+      if (st->cnt > p.cand_cap - 32 * Core::CHUNK_WORDS) cut_exact(p.k);
     }
   });
 }
@@ -517,14 +506,30 @@ struct FusedLaunch {
   template <int G, int b, int W>
   kvs_status operator()() const {
     using Core = ScanCore<G, b, W>;
-    const size_t extra = 2048 * sizeof(unsigned) + sizeof(SegState);
-    const size_t smem = Core::smem_bytes(p.nsets, extra);
-    auto kern = fathom_scan_topk_kernel<G, b, W>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    const size_t base_extra = 2048 * sizeof(unsigned) + sizeof(SegState);
+    const int chunk_keys = 32 * Core::CHUNK_WORDS;
+    // keys in shared memory when 2k + one chunk of them fit beside two stages
+    const int cap_s = 2 * p.k + chunk_keys;
+    const size_t extra_s = base_extra + static_cast<size_t>(cap_s) * sizeof(uint32_t);
     ScanParams q = p;
     q.warps = W;
-    q.nstage = Core::nstages(p.nsets, extra);
-    kern<<<grid, Core::THREADS, smem, s>>>(q);
+    if (Core::nstages(p.nsets, extra_s) >= 2) {
+      q.cand_cap = cap_s;
+      q.trim_at = 2 * p.k;
+      q.nstage = Core::nstages(p.nsets, extra_s);
+      const size_t smem = Core::smem_bytes(p.nsets, extra_s);
+      auto kern = fathom_scan_topk_kernel<G, b, W, true>;
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      kern<<<grid, Core::THREADS, smem, s>>>(q);
+    } else {
+      q.cand_cap = kCandCap;
+      q.trim_at = kCandCap - chunk_keys;
+      q.nstage = Core::nstages(p.nsets, base_extra);
+      const size_t smem = Core::smem_bytes(p.nsets, base_extra);
+      auto kern = fathom_scan_topk_kernel<G, b, W, false>;
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      kern<<<grid, Core::THREADS, smem, s>>>(q);
+    }
     return check_launch("decode_step(scan+topk)");
   }
 };
@@ -539,8 +544,8 @@ bool fused_topk_supported(int n_max, int k, int B) {
 size_t fused_ws_bytes(int RG, int n_max, int k, int B) {
   const Layout L = fused_layout(RG, n_max, k, B);
   WsCarver c(nullptr);
-  c.take<uint32_t>(static_cast<size_t>(L.grid) * 2 * kCandCap);
-  c.take<int32_t>(static_cast<size_t>(L.grid) * 2 * kCandCap);
+  c.take<uint32_t>(static_cast<size_t>(L.grid) * kCandCap);
+  c.take<int32_t>(static_cast<size_t>(L.grid) * kCandCap);
   c.take<uint64_t>(static_cast<size_t>(L.grid) * kCandCap);
   c.take<uint32_t>(static_cast<size_t>(RG) * L.segs * L.seg_cap);
   c.take<int32_t>(static_cast<size_t>(RG) * L.segs * L.seg_cap);
@@ -558,8 +563,8 @@ kvs_status fathom_scan_topk_launch(ScanParams p, void* ws, const int32_t* slot_m
   p.segs_per_row = L.segs;
   p.seg_cap = L.seg_cap;
   WsCarver c(ws);
-  p.cbuf_key = c.take<uint32_t>(static_cast<size_t>(L.grid) * 2 * kCandCap);
-  p.cbuf_idx = c.take<int32_t>(static_cast<size_t>(L.grid) * 2 * kCandCap);
+  p.cbuf_key = c.take<uint32_t>(static_cast<size_t>(L.grid) * kCandCap);
+  p.cbuf_idx = c.take<int32_t>(static_cast<size_t>(L.grid) * kCandCap);
   p.cbuf_comp = c.take<uint64_t>(static_cast<size_t>(L.grid) * kCandCap);
   p.cand_key = c.take<uint32_t>(static_cast<size_t>(p.RG) * L.segs * L.seg_cap);
   p.cand_idx = c.take<int32_t>(static_cast<size_t>(p.RG) * L.segs * L.seg_cap);
