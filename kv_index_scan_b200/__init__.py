@@ -154,6 +154,39 @@ class FathomIndex:
                             self.D, self.W, int(self.host_mapped))
 
 
+class MappedHostIndex(FathomIndex):
+    """A FathomIndex whose planes live in mapped pinned host memory
+    (cudaHostAlloc with cudaHostAllocMapped); the scan reads them over the host
+    link through the device alias from cudaHostGetDevicePointer. The host
+    buffer is freed when this object is."""
+
+    def __init__(self, index: FathomIndex):
+        from cuda.bindings import runtime as rt
+        self._rt = rt
+        nbytes = index.planes.numel() * 4
+        err, hptr = rt.cudaHostAlloc(nbytes, rt.cudaHostAllocMapped | rt.cudaHostAllocPortable)
+        if err != rt.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"cudaHostAlloc: {err}")
+        self._hptr = hptr
+        err, dptr = rt.cudaHostGetDevicePointer(hptr, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"cudaHostGetDevicePointer: {err}")
+        torch.cuda.synchronize()
+        err, = rt.cudaMemcpy(hptr, index.planes.data_ptr(), nbytes,
+                             rt.cudaMemcpyKind.cudaMemcpyDeviceToHost)
+        if err != rt.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"cudaMemcpy: {err}")
+        super().__init__(index.planes, index.kmin, index.kstep, index.kvar, planes_ptr=int(dptr),
+                         host_mapped=True)
+        self.nbytes = nbytes
+
+    def __del__(self):
+        try:
+            self._rt.cudaFreeHost(self._hptr)
+        except Exception:
+            pass
+
+
 class Plan:
     """Per-(r, g) bit allocation: t u8 [R][G][D], plane_idx int16 [R][G][B]
     (u16 plane ids c*4+p), plane_w f32 [R][G][B], C f32 [R][G]."""

@@ -180,9 +180,10 @@ struct ScanCore {
   static constexpr int TBL_BYTES = (1 << b) * 128;
   static constexpr int STAGE_BYTES = NPOS * ROW_BYTES;
 
-  // layout: [tables | nstage stages | 256 bytes of barriers | extra]
+  // layout: [tables | nstage stages | 256 bytes of barriers | extra], within
+  // the 227 KB of dynamic shared memory a block may opt in to on sm_100
   static int nstages(int nsets, size_t extra = 0) {
-    const int budget = 224 * 1024 - nsets * TBL_BYTES - 256 - static_cast<int>(extra);
+    const int budget = 227 * 1024 - nsets * TBL_BYTES - 256 - static_cast<int>(extra);
     const int s = budget / STAGE_BYTES;
     return s > 4 ? 4 : s;
   }

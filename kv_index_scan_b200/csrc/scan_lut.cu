@@ -10,11 +10,12 @@
 // ALUs deliver per HBM byte (about 0.7 operations per plane bit at full HBM
 // bandwidth). This kernel does it in about one:
 //
-//  * Staging. A producer warp copies, for a chunk of 128 words (4096 keys) of
-//    one (request, KV head) row, the planes of one "table set" into a shared
-//    memory stage with 1-D TMA bulk copies (cp.async.bulk, 512 bytes per
-//    plane), completing on the stage's mbarrier. Stages form a ring; consumer
-//    warps release a stage when done with it. Every wait is bounded.
+//  * Staging. A producer warp copies, for a chunk of 16 words per consumer
+//    warp (192 words, 6,144 keys, with 12 consumer warps) of one (request, KV
+//    head) row, the planes of one "table set" into a shared memory stage with
+//    1-D TMA bulk copies (cp.async.bulk, one per plane), completing on the
+//    stage's mbarrier. Stages form a ring; consumer warps release a stage when
+//    done with it. Every wait is bounded.
 //  * Transpose. Two consumer threads share a 32-key word, 16 keys each. A
 //    thread loads its 16-bit half of 32 plane words (conflict-free 2-byte
 //    reads), pairs planes k and k + 16 in one register, and finishes the

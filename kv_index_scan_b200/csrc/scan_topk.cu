@@ -51,43 +51,50 @@ __host__ __device__ __forceinline__ int block_of_chunk(long long x, long long C,
   return b;
 }
 
-// Warp 0 of a group: in a histogram over [0, nbins) bins, the bin holding
-// rank krem counted from the top; returns the bin and the count above it.
-__device__ __forceinline__ void find_bin_from_top(const unsigned* hist, int nbins, int krem,
-                                                  int& bin, int& above_out) {
-  const int lane = threadIdx.x & 31;
-  int above = 0;
-  bin = 0;
-  above_out = 0;
-  for (int top = nbins; top > 0; top -= 64) {
-    const int b0 = top - 1 - 2 * lane, b1 = b0 - 1;
-    const int c0 = b0 >= 0 ? static_cast<int>(hist[b0]) : 0;
-    const int c1 = b1 >= 0 ? static_cast<int>(hist[b1]) : 0;
-    const int mine = c0 + c1;
-    int incl = mine;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-      if (lane >= d) incl += o;
-    }
-    const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-    if (above + total >= krem) {
-      const unsigned hit = __ballot_sync(0xFFFFFFFFu, above + incl >= krem);
-      const int l = __ffs(hit) - 1;
-      const int ex = __shfl_sync(0xFFFFFFFFu, incl - mine, l);
-      const int cb0 = __shfl_sync(0xFFFFFFFFu, c0, l);
-      const int bb0 = top - 1 - 2 * l;
-      if (above + ex + cb0 >= krem) {
-        bin = bb0;
-        above_out = above + ex;
-      } else {
-        bin = bb0 - 1;
-        above_out = above + ex + cb0;
-      }
-      return;
-    }
-    above += total;
+// Group-wide (all nthreads threads, uniform call): in a histogram over
+// [0, nbins) bins, the bin holding rank krem counted from the top, and the
+// count above it, into res[0], res[1]. Each thread sums a run of bins, one
+// exclusive scan over the threads finds the run holding the rank, and its
+// thread walks it. wsum holds one entry per warp. Ends with a barrier.
+template <typename Sync>
+__device__ void find_bin_from_top(const unsigned* hist, int nbins, int krem, int* wsum, int* res,
+                                  int tid, int nthreads, Sync sync) {
+  const int per = (nbins + nthreads - 1) / nthreads;
+  const int hi = nbins - tid * per;  // this thread's bins: hi - 1 down to hi - per
+  int mine = 0;
+  for (int e = 0; e < per; ++e) {
+    const int bb = hi - 1 - e;
+    if (bb >= 0) mine += static_cast<int>(hist[bb]);
   }
+  const int lane = tid & 31, warp = tid >> 5;
+  int incl = mine;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+    if (lane >= d) incl += o;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  if (tid == 0) {
+    res[0] = 0;
+    res[1] = 0;
+  }
+  sync();
+  const int before = __reduce_add_sync(0xFFFFFFFFu, lane < warp ? wsum[lane] : 0);
+  const int ex = before + incl - mine;
+  if (mine > 0 && ex < krem && ex + mine >= krem) {
+    int above = ex;
+    for (int e = 0; e < per && hi - 1 - e >= 0; ++e) {
+      const int bb = hi - 1 - e;
+      const int c = static_cast<int>(hist[bb]);
+      if (above + c >= krem) {
+        res[0] = bb;
+        res[1] = above;
+        break;
+      }
+      above += c;
+    }
+  }
+  sync();
 }
 
 __device__ __forceinline__ void hist_add(unsigned* hist, int bin) {
@@ -100,6 +107,7 @@ struct SelectState {
   unsigned long long prefix, mask;
   int krem;
   uint32_t tau;
+  int wsum[32], res[2];
 };
 
 // Group-wide: the kk-th largest of the n distinct 53-bit composites in src
@@ -135,14 +143,12 @@ __device__ uint64_t select_kth_composite(const uint64_t* src, int n, int kk, uns
       }
     }
     sync();
-    if (tid < 32) {
-      int bin, above;
-      find_bin_from_top(hist, static_cast<int>(dmask) + 1, st->krem, bin, above);
-      if (tid == 0) {
-        st->prefix = prefix | (static_cast<unsigned long long>(bin) << shift);
-        st->mask = mask | (static_cast<unsigned long long>(dmask) << shift);
-        st->krem -= above;
-      }
+    find_bin_from_top(hist, static_cast<int>(dmask) + 1, st->krem, st->wsum, st->res, tid,
+                      nthreads, sync);
+    if (tid == 0) {
+      st->prefix = prefix | (static_cast<unsigned long long>(st->res[0]) << shift);
+      st->mask = mask | (static_cast<unsigned long long>(dmask) << shift);
+      st->krem -= st->res[1];
     }
     sync();
   }
@@ -193,16 +199,9 @@ __global__ void KVS_SCAN_BOUNDS(G, b, W) fathom_scan_topk_kernel(ScanParams p) {
         hist_add(hist, base + e * NT + t < n ? static_cast<int>(kv[e] >> 21) : -1);
     }
     sync();
-    if (t < 32) {
-      int bin, above;
-      find_bin_from_top(hist, 2048, kk, bin, above);
-      if (t == 0) {
-        st->sel.tau = static_cast<uint32_t>(bin);
-        st->sel.krem = kk - above;
-      }
-    }
-    sync();
-    const uint32_t b1 = st->sel.tau;
+    find_bin_from_top(hist, 2048, kk, st->sel.wsum, st->sel.res, t, NT, sync);
+    const uint32_t b1 = static_cast<uint32_t>(st->sel.res[0]);
+    const int krem = kk - st->sel.res[1];
     for (int bb = t; bb < 2048; bb += NT) hist[bb] = 0;
     sync();
     for (int base = 0; base < n; base += 4 * NT) {
@@ -219,42 +218,47 @@ __global__ void KVS_SCAN_BOUNDS(G, b, W) fathom_scan_topk_kernel(ScanParams p) {
       }
     }
     sync();
-    if (t < 32) {
-      int bin, above;
-      find_bin_from_top(hist, 2048, st->sel.krem, bin, above);
-      if (t == 0) st->sel.tau = (b1 << 21) | (static_cast<uint32_t>(bin) << 10);
-    }
-    sync();
-    return st->sel.tau;
+    find_bin_from_top(hist, 2048, krem, st->sel.wsum, st->sel.res, t, NT, sync);
+    return (b1 << 21) | (static_cast<uint32_t>(st->sel.res[0]) << 10);
   };
 
   // Keep the held entries with key >= tau, compacted in place: each round
-  // reads one entry per thread, then (after a barrier) writes the kept ones
-  // below it, so no unread entry is ever overwritten (uniform call).
+  // reads kRound entries per thread (their index loads in flight together),
+  // then (after a barrier) writes the kept ones below them, so no unread
+  // entry is ever overwritten (uniform call).
   auto keep_at_least = [&](uint32_t tau, float tau_f) {
+    constexpr int kRound = 8;
     const int t = threadIdx.x;
     const int n = st->cnt;
     if (t == 0) st->cnt2 = 0;
     sync();
-    for (int base = 0; base < n; base += NT) {
-      const int i = base + t;
-      uint32_t key = 0u;
-      int32_t ix = 0;
-      if (i < n) {
-        key = kb[i];
-        ix = ib[i];
+    for (int base = 0; base < n; base += kRound * NT) {
+      uint32_t key[kRound];
+      int32_t ix[kRound];
+#pragma unroll
+      for (int e = 0; e < kRound; ++e) {
+        const int i = base + e * NT + t;
+        key[e] = i < n ? kb[i] : 0u;
       }
-      const bool take = i < n && key >= tau;
+#pragma unroll
+      for (int e = 0; e < kRound; ++e) {
+        const int i = base + e * NT + t;
+        ix[e] = (i < n && key[e] >= tau) ? ib[i] : 0;
+      }
       sync();
-      const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
-      if (m) {
+#pragma unroll
+      for (int e = 0; e < kRound; ++e) {
+        const int i = base + e * NT + t;
+        const bool take = i < n && key[e] >= tau;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
+        if (m == 0u) continue;
         const int lane = t & 31, leader = __ffs(m) - 1;
         int pos = 0;
         if (lane == leader) pos = atomicAdd(&st->cnt2, __popc(m));
         pos = __shfl_sync(0xFFFFFFFFu, pos, leader) + __popc(m & ((1u << lane) - 1u));
         if (take) {
-          kb[pos] = key;
-          ib[pos] = ix;
+          kb[pos] = key[e];
+          ib[pos] = ix[e];
         }
       }
     }
@@ -310,9 +314,43 @@ __global__ void KVS_SCAN_BOUNDS(G, b, W) fathom_scan_topk_kernel(ScanParams p) {
     keep_at_least(tau, key_to_float(tau));
   };
 
+  // A threshold for a segment's first chunk from the chunk's own scores (in
+  // registers), when it holds at least k valid keys: the lower edge of the
+  // 22-bit key cell holding its k-th largest key (uniform call).
+  auto chunk_threshold = [&](int i0, int nr, const float (&acc)[kKeysPerThread]) {
+    const int t = threadIdx.x;
+    uint32_t key[kKeysPerThread];
+#pragma unroll
+    for (int j = 0; j < kKeysPerThread; ++j) key[j] = ordered_key(acc[j]);
+    for (int bb = t; bb < 2048; bb += NT) hist[bb] = 0;
+    sync();
+#pragma unroll
+    for (int j = 0; j < kKeysPerThread; ++j)
+      hist_add(hist, i0 + j < nr ? static_cast<int>(key[j] >> 21) : -1);
+    sync();
+    find_bin_from_top(hist, 2048, p.k, st->sel.wsum, st->sel.res, t, NT, sync);
+    const uint32_t b1 = static_cast<uint32_t>(st->sel.res[0]);
+    const int krem = p.k - st->sel.res[1];
+    for (int bb = t; bb < 2048; bb += NT) hist[bb] = 0;
+    sync();
+#pragma unroll
+    for (int j = 0; j < kKeysPerThread; ++j)
+      hist_add(hist, (i0 + j < nr && (key[j] >> 21) == b1) ? static_cast<int>((key[j] >> 10) & 2047u)
+                                                            : -1);
+    sync();
+    find_bin_from_top(hist, 2048, krem, st->sel.wsum, st->sel.res, t, NT, sync);
+    const uint32_t tau = (b1 << 21) | (static_cast<uint32_t>(st->sel.res[0]) << 10);
+    if (t == 0) {
+      st->tau_set = 1;
+      st->tau_f = key_to_float(tau);
+    }
+    sync();
+  };
+
   core.run([&](int u, int c, int nr, const float (&acc)[kKeysPerThread], int t) {
     // 1. keys at or above the running threshold join the segment's candidates
     const int i0 = 32 * (c * Core::CHUNK_WORDS + (t >> 1)) + kKeysPerThread * (t & 1);
+    if (st->tau_set == 0 && nr - 32 * c * Core::CHUNK_WORDS >= p.k) chunk_threshold(i0, nr, acc);
     const bool has_tau = st->tau_set != 0;
     const float tau = st->tau_f;
 #pragma unroll
@@ -343,6 +381,7 @@ __global__ void KVS_SCAN_BOUNDS(G, b, W) fathom_scan_topk_kernel(ScanParams p) {
       const int slot = static_cast<int>(blockIdx.x) -
                        block_of_chunk(static_cast<long long>(u) * p.chunks_per_row, C, gridDim.x);
       const size_t off = (static_cast<size_t>(u) * p.segs_per_row + slot) * p.seg_cap;
+#pragma unroll 4
       for (int e = threadIdx.x; e < kk; e += NT) {
         p.cand_key[off + e] = kb[e];
         p.cand_idx[off + e] = ib[e];
@@ -443,7 +482,7 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(
     keys[e] = i < nchosen ? chosen[i] : 0xFFFFFFFFu;
   }
   __syncthreads();
-  Sort(sm.sort).Sort(keys);
+  Sort(sm.sort).Sort(keys, 0, kIdxBits);  // indices < 2^21; the pad sorts last (stable)
   int my_miss = 0;
 #pragma unroll
   for (int e = 0; e < kMergeItems; ++e) {

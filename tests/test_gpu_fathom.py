@@ -274,3 +274,29 @@ def test_decode_step_all_scores_tied_takes_first_indices(kvs):
     torch.cuda.synchronize()
     assert torch.equal(step.idx.cpu(), torch.arange(k, dtype=torch.int32).expand(R, G, k))
     assert torch.all(step.misses == k)
+
+
+@pytest.mark.parametrize("B", [68, 92])
+def test_host_mapped_index_scan_and_decode(kvs, B):
+    """The index planes in mapped pinned host memory, read over the host link
+    by the same call: scores within the f32 bound of the oracle, and the same
+    selection as the oracle (up to ties inside the band)."""
+    R, G, n = 2, 2, 20000
+    K, V, nl = synth.fathom_kv(R, G, D, n, seed=61)
+    q = synth.queries(R, G, 4, D, seed=61)
+    ix = kvs.build_fathom_index(K.to(DEV), nl)
+    hix = kvs.MappedHostIndex(ix)
+    plan = kvs.fathom_plan_bits(q.to(DEV), hix, B)
+    sc = kvs.index_scan_fathom(hix, plan, nl, n).cpu().numpy()
+    step = kvs.DecodeStep(hix, nl, n, 4, B, 512, K.to(DEV), V.to(DEV))
+    step(q.to(DEV))
+    torch.cuda.synchronize()
+    planes, kmin, kstep, kvar = oracle.build_index_batch(K, nl, kvs.plane_words(n))
+    ref = oracle.decode_batch(q, planes, kmin, kstep, kvar, nl, B, 512, None, None, None, K, V,
+                              1 / math.sqrt(D), want_scores=True)
+    for r in range(R):
+        for g in range(G):
+            t, qbar = oracle.plan_bits(q[r, g], kvar[r, g], B)
+            tol = fathom_score_tol(qbar, kmin[r, g], kstep[r, g], B)
+            assert np.max(np.abs(sc[r, g] - ref["scores"][r, g])) <= tol
+            check_selection(step.idx[r, g].cpu().numpy(), ref["idx"][r, g], ref["scores"][r, g], 512)

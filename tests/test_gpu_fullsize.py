@@ -1,0 +1,91 @@
+"""Full-size parity: the 128K decode layer (16 requests x 8 KV heads x 131072
+keys, B in {68, 92, 136, 512}, top-2048, 4096 hot slots) and the 1M layer
+(4 x 8 x 1048576, B in {92, 136}) in the launch configuration the benchmark
+times, checked on sampled (request, KV head) rows that the oracle computes
+one by one.
+
+Inputs are drawn on the GPU by the seeded generator and copied row by row to
+the host for the oracle. The hot buffers of the sampled rows are built around
+the oracle's own selection (20% of it missing); the other rows get hot buffers
+around a random selection, which only changes their hit pattern.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests._parity import ATTN_TOL, check_selection
+
+pytestmark = pytest.mark.gpu
+D, H = 128, 4
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def kvs():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import kv_index_scan_b200
+    return kv_index_scan_b200
+
+
+def _np16(t):
+    return t.detach().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def _run_sampled(kvs, R, G, n, B, k, S, rows, seed):
+    K, V, nl = synth.fathom_kv(R, G, D, n, seed=seed, device=DEV)
+    q = synth.queries(R, G, H, D, seed=seed, device=DEV)
+    W = kvs.plane_words(n)
+    scale = 1 / math.sqrt(D)
+    # oracle on the sampled rows: its own index, plan, scan and selection
+    sel = np.stack([np.sort(np.random.default_rng(seed + u).choice(n, k, replace=False))
+                    for u in range(R * G)]).reshape(R, G, k).astype(np.int32)
+    ref = {}
+    for u in rows:
+        r, g = divmod(u, G)
+        Kr = K[r, g].cpu().unsqueeze(0).unsqueeze(0)
+        Vr = V[r, g].cpu().unsqueeze(0).unsqueeze(0)
+        qr = q[r, g].cpu().unsqueeze(0).unsqueeze(0)
+        planes, kmin, kstep, kvar = oracle.build_index_batch(Kr, [n], W)
+        res = oracle.decode_batch(qr, planes, kmin, kstep, kvar, [n], B, k, None, None, None, Kr,
+                                  Vr, scale, want_scores=True)
+        sel[r, g] = res["idx"][0, 0]
+        ref[u] = dict(planes=planes[0, 0], kvar=kvar[0, 0], t=res["t"][0, 0], idx=res["idx"][0, 0],
+                      scores=res["scores"][0, 0], K=Kr, V=Vr, q=qr, index=(planes, kmin, kstep, kvar))
+    slot_map, hot_tok = synth.slot_map_from_selection(sel, nl, n, S, 0.2, seed=seed)
+    hotK, hotV = synth.hot_rows(K, hot_tok), synth.hot_rows(V, hot_tok)
+    ix = kvs.build_fathom_index(K, nl, W)
+    step = kvs.DecodeStep(ix, nl, n, H, B, k, K, V, torch.from_numpy(slot_map).to(DEV), hotK, hotV)
+    step(q)
+    torch.cuda.synchronize()
+    for u in rows:
+        r, g = divmod(u, G)
+        e = ref[u]
+        # the index rows are bit-exact
+        assert np.array_equal(ix.planes[r, g].cpu().numpy().view(np.uint32), e["planes"])
+        assert np.array_equal(ix.kvar[r, g].cpu().numpy(), e["kvar"])
+        assert np.array_equal(step.plan.t[r, g].cpu().numpy(), e["t"])
+        d = check_selection(step.idx[r, g].cpu().numpy(), e["idx"], e["scores"], k)
+        # the oracle's attention and misses over the same slot map
+        planes, kmin, kstep, kvar = e["index"]
+        res = oracle.decode_batch(e["q"], planes, kmin, kstep, kvar, [n], B, k,
+                                  slot_map[r, g][None, None], hotK[r, g].cpu()[None, None],
+                                  hotV[r, g].cpu()[None, None], e["K"], e["V"], scale)
+        if d == 0:
+            assert np.array_equal(step.slots[r, g].cpu().numpy(), res["slots"][0, 0])
+            assert int(step.misses[r, g]) == int(res["misses"][0, 0]) == round(0.2 * k)
+            assert np.max(np.abs(step.out[r, g].cpu().numpy() - res["out"][0, 0])) < ATTN_TOL
+
+
+@pytest.mark.parametrize("B", [92, 68, 136, 512])
+def test_decode_step_128k_layer_sampled_rows(kvs, B):
+    _run_sampled(kvs, 16, 8, 131072, B, 2048, 4096, rows=[0, 37, 127], seed=100 + B)
+
+
+@pytest.mark.parametrize("B", [92, 136])
+def test_decode_step_1m_layer_sampled_rows(kvs, B):
+    _run_sampled(kvs, 4, 8, 1048576, B, 2048, 4096, rows=[5, 31], seed=200 + B)
