@@ -10,8 +10,10 @@
 // the B largest "bit events" (c, j), value w_c 4^-j, in the order
 // (value desc, c asc, j asc). Every event gets a distinct 64-bit key -- the bit
 // pattern of the exact double w_c 4^-j (an f32 widened to fp64 has 29 zero low
-// mantissa bits) with 511 - (4c + j) in the low bits -- and an event is taken
-// when fewer than B keys exceed its own. One 512-thread block per (r, g).
+// mantissa bits) with 511 - (4c + j) in the low bits -- and the events whose
+// keys are among the B largest are taken: a bitonic sort of the 512 keys in
+// shared memory (descending), the first B of it marked. One 512-thread block
+// per (r, g).
 #include "internal.cuh"
 
 namespace kvs {
@@ -28,6 +30,7 @@ __global__ void __launch_bounds__(512) plan_bits_kernel(
   __shared__ float qb[kD], wv[kD];
   __shared__ unsigned long long key[4 * kD];
   __shared__ int tcount[kD], start[kD];
+  __shared__ unsigned char took[4 * kD];
   __shared__ float cterm[kD];
   if (tid < kD) {
     const float* qq = q + static_cast<size_t>(u) * H * kD;
@@ -45,12 +48,28 @@ __global__ void __launch_bounds__(512) plan_bits_kernel(
     key[tid] = static_cast<unsigned long long>(__double_as_longlong(v)) |
                static_cast<unsigned long long>(511 - tid);
   }
+  took[tid] = 0;
   __syncthreads();
-  const unsigned long long mine = key[tid];
-  int rank = 0;
-#pragma unroll 8
-  for (int e = 0; e < 4 * kD; ++e) rank += key[e] > mine ? 1 : 0;
-  const bool taken = rank < B;
+  // bitonic sort, descending: thread tid < 256 owns one compare-exchange pair
+  // per stage
+  for (int size = 2; size <= 4 * kD; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (tid < 2 * kD) {
+        const int lo = 2 * tid - (tid & (stride - 1));
+        const int hi = lo + stride;
+        const bool desc = (lo & size) == 0;
+        const unsigned long long a = key[lo], b = key[hi];
+        if ((a < b) == desc) {
+          key[lo] = b;
+          key[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  if (tid < B) took[511 - static_cast<int>(key[tid] & 511ull)] = 1;
+  __syncthreads();
+  const bool taken = took[tid] != 0;
   const unsigned ball = __ballot_sync(0xFFFFFFFFu, taken);
   const int tc = __popc((ball >> ((tid & 31) & ~3)) & 0xFu);
   if (j == 0) {

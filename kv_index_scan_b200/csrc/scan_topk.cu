@@ -19,11 +19,9 @@
 //
 // Merge kernel: one block per row gathers its segments' candidates as
 // distinct 53-bit composites (score key << 21 | (2^21 - 1 - index)), selects
-// exactly the k largest (five radix passes), sorts their indices ascending
-// (block radix sort), writes idx, and looks every selected key up in the
+// exactly the k largest (radix passes), emits their indices in ascending order
+// through a bitmap over the row, and looks every selected key up in the
 // hot-buffer slot map (slots; misses = the number absent from the hot buffer).
-#include <cub/block/block_radix_sort.cuh>
-
 #include "internal.cuh"
 #include "scan_core.cuh"
 
@@ -105,26 +103,27 @@ __device__ __forceinline__ void hist_add(unsigned* hist, int bin) {
 
 struct SelectState {
   unsigned long long prefix, mask;
-  int krem;
+  int krem, done;
   uint32_t tau;
   int wsum[32], res[2];
 };
 
 // Group-wide: the kk-th largest of the n distinct 53-bit composites in src
-// (kk >= 1, n >= kk); five radix passes of 11/11/11/10/10 bits.
+// (kk >= 1, n >= kk); radix passes of 11/11/11/10/10 bits, stopping early once
+// the bin holding the rank is taken whole (its lower edge then selects exactly
+// kk: usually after the third pass, which resolves the full score key).
 template <typename Sync>
 __device__ uint64_t select_kth_composite(const uint64_t* src, int n, int kk, unsigned* hist,
                                          SelectState* st, int tid, int nthreads, Sync sync) {
-  const int shifts[5] = {42, 31, 20, 10, 0};
-  const int widths[5] = {11, 11, 11, 10, 10};
   if (tid == 0) {
     st->prefix = 0ull;
     st->mask = 0ull;
     st->krem = kk;
+    st->done = 0;
   }
   for (int pass = 0; pass < 5; ++pass) {
-    const int shift = shifts[pass];
-    const unsigned dmask = (1u << widths[pass]) - 1u;
+    const int shift = pass < 3 ? 42 - 11 * pass : (pass == 3 ? 10 : 0);
+    const unsigned dmask = pass < 3 ? 2047u : 1023u;
     for (int b = tid; b < 2048; b += nthreads) hist[b] = 0;
     sync();
     const unsigned long long prefix = st->prefix, mask = st->mask;
@@ -146,11 +145,14 @@ __device__ uint64_t select_kth_composite(const uint64_t* src, int n, int kk, uns
     find_bin_from_top(hist, static_cast<int>(dmask) + 1, st->krem, st->wsum, st->res, tid,
                       nthreads, sync);
     if (tid == 0) {
-      st->prefix = prefix | (static_cast<unsigned long long>(st->res[0]) << shift);
+      const int bin = st->res[0];
+      st->prefix = prefix | (static_cast<unsigned long long>(bin) << shift);
       st->mask = mask | (static_cast<unsigned long long>(dmask) << shift);
       st->krem -= st->res[1];
+      st->done = st->krem == static_cast<int>(hist[bin]) ? 1 : 0;
     }
     sync();
+    if (st->done) break;
   }
   return st->prefix;
 }
@@ -353,20 +355,29 @@ __global__ void KVS_SCAN_BOUNDS(G, b, W) fathom_scan_topk_kernel(ScanParams p) {
     if (st->tau_set == 0 && nr - 32 * c * Core::CHUNK_WORDS >= p.k) chunk_threshold(i0, nr, acc);
     const bool has_tau = st->tau_set != 0;
     const float tau = st->tau_f;
+    // one shared-memory atomic per warp and chunk: the warp's takes are
+    // counted first, then written at ballot-ordered positions
+    const int lane = threadIdx.x & 31;
+    const unsigned lt = (1u << lane) - 1u;
+    unsigned m[kKeysPerThread];
+    int wtotal = 0;
 #pragma unroll
     for (int j = 0; j < kKeysPerThread; ++j) {
-      const int i = i0 + j;
-      const bool take = i < nr && (!has_tau || acc[j] >= tau);
-      const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
-      if (m == 0u) continue;
-      const int lane = threadIdx.x & 31;
-      const int leader = __ffs(m) - 1;
+      m[j] = __ballot_sync(0xFFFFFFFFu, i0 + j < nr && (!has_tau || acc[j] >= tau));
+      wtotal += __popc(m[j]);
+    }
+    if (wtotal > 0) {
       int base = 0;
-      if (lane == leader) base = atomicAdd(&st->cnt, __popc(m));
-      base = __shfl_sync(0xFFFFFFFFu, base, leader) + __popc(m & ((1u << lane) - 1u));
-      if (take) {
-        kb[base] = ordered_key(acc[j]);
-        ib[base] = i;
+      if (lane == 0) base = atomicAdd(&st->cnt, wtotal);
+      base = __shfl_sync(0xFFFFFFFFu, base, 0);
+#pragma unroll
+      for (int j = 0; j < kKeysPerThread; ++j) {
+        if ((m[j] >> lane) & 1u) {
+          const int pos = base + __popc(m[j] & lt);
+          kb[pos] = ordered_key(acc[j]);
+          ib[pos] = i0 + j;
+        }
+        base += __popc(m[j]);
       }
     }
     sync();
@@ -399,31 +410,34 @@ __global__ void KVS_SCAN_BOUNDS(G, b, W) fathom_scan_topk_kernel(ScanParams p) {
   });
 }
 
-// One block per (r, g): gather the segments' candidates, select, sort, slot
-// lookup. 1024 threads, up to 4096 selected.
+// One block per (r, g): gather the segments' candidates, select the k best,
+// emit their indices in ascending order, look up their slots. 1024 threads.
+// The ascending order comes from a bitmap over the row's key indices (in the
+// workspace): the selected keys set their bits, each thread counts the bits
+// of its run of words, one block-wide scan gives every thread its output
+// position, and the threads write the set bits of their runs in order.
 constexpr int kMergeThreads = 1024;
-constexpr int kMergeItems = 4;
+constexpr int kMergeMaxK = 4096;
 constexpr int kMergeSmemEntries = 20480;
+static_assert(kMergeThreads == 32 * 32, "the merge sums its per-warp counts with one warp");
+
+__host__ __device__ __forceinline__ int bitmap_words(int n_max) {
+  return (((n_max + 31) / 32) + 3) & ~3;
+}
 
 __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(
-    ScanParams p, int scan_grid, uint64_t* __restrict__ gscratch,
+    ScanParams p, int scan_grid, uint64_t* __restrict__ gscratch, uint32_t* __restrict__ bitmap,
     const int32_t* __restrict__ slot_map, int32_t* __restrict__ idx, int32_t* __restrict__ slots,
     int32_t* __restrict__ misses) {
-  using Sort = cub::BlockRadixSort<uint32_t, kMergeThreads, kMergeItems>;
-  // the select's histogram, the chosen indices and the sort's scratch are
-  // used one after another, separated by barriers: one union
-  __shared__ union {
-    unsigned hist[2048];
-    uint32_t chosen[kMergeThreads * kMergeItems];
-    typename Sort::TempStorage sort;
-  } sm;
+  __shared__ unsigned hist[2048];
   __shared__ SelectState sel;
   __shared__ int seg_count[64], seg_off[65];
-  __shared__ int nsel;
+  __shared__ int wsum[kMergeThreads / 32];
   __shared__ int miss_warp[kMergeThreads / 32];
   extern __shared__ __align__(16) uint64_t comp_smem[];
   const int u = blockIdx.x;
   const int t = threadIdx.x;
+  const int lane = t & 31, warp = t >> 5;
   const int nr = p.n[u / p.Gheads];
   const int kk = min(p.k, nr);
   const long long C = static_cast<long long>(p.RG) * p.chunks_per_row;
@@ -439,57 +453,95 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(
       o += seg_count[s];
     }
     seg_off[segs] = o;
-    nsel = 0;
   }
+  // clear this row's bitmap meanwhile
+  const int words = bitmap_words(p.n_max);
+  uint32_t* bm = bitmap + static_cast<size_t>(u) * words;
+  for (int w = 4 * t; w < words; w += 4 * kMergeThreads)
+    *reinterpret_cast<uint4*>(bm + w) = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
   const int total = seg_off[segs];
   uint64_t* comp = total <= kMergeSmemEntries
                        ? comp_smem
                        : gscratch + static_cast<size_t>(u) * p.segs_per_row * p.seg_cap;
-  for (int s = 0; s < segs; ++s) {
-    const size_t off = (static_cast<size_t>(u) * p.segs_per_row + s) * p.seg_cap;
-    for (int i = t; i < seg_count[s]; i += kMergeThreads)
-      comp[seg_off[s] + i] = make_composite(p.cand_key[off + i], p.cand_idx[off + i]);
+  // gather the candidates as composites, four loads in flight per thread
+  for (int base = 0; base < total; base += 4 * kMergeThreads) {
+    uint32_t key[4];
+    int32_t ix[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int f = base + e * kMergeThreads + t;
+      key[e] = 0u;
+      ix[e] = 0;
+      if (f < total) {
+        int s = 0;
+        while (f >= seg_off[s + 1]) ++s;
+        const size_t off = (static_cast<size_t>(u) * p.segs_per_row + s) * p.seg_cap + (f - seg_off[s]);
+        key[e] = p.cand_key[off];
+        ix[e] = p.cand_idx[off];
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int f = base + e * kMergeThreads + t;
+      if (f < total) comp[f] = make_composite(key[e], ix[e]);
+    }
   }
   __syncthreads();
   uint64_t tau = 0ull;
   if (kk > 0 && total > kk)
-    tau = select_kth_composite(comp, total, kk, sm.hist, &sel, t, kMergeThreads,
+    tau = select_kth_composite(comp, total, kk, hist, &sel, t, kMergeThreads,
                                [] { __syncthreads(); });
-  __syncthreads();
-  // the selected indices, unordered, into the blocked sort input
-  uint32_t* chosen = sm.chosen;
-  for (int base = 0; base < total; base += kMergeThreads) {
-    const int i = base + t;
-    const uint64_t c = i < total ? comp[i] : 0ull;
-    const bool take = kk > 0 && i < total && c >= tau;
-    const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
-    if (m) {
-      const int lane = t & 31, leader = __ffs(m) - 1;
-      int basew = 0;
-      if (lane == leader) basew = atomicAdd(&nsel, __popc(m));
-      basew = __shfl_sync(0xFFFFFFFFu, basew, leader);
-      const int pos = basew + __popc(m & ((1u << lane) - 1u));
-      if (take && pos < kMergeThreads * kMergeItems) chosen[pos] = composite_index(c);
+  // the selected keys set their bits
+  if (kk > 0) {
+    for (int f = t; f < total; f += kMergeThreads) {
+      const uint64_t c = comp[f];
+      if (c >= tau) {
+        const int i = composite_index(c);
+        atomicOr(bm + (i >> 5), 1u << (i & 31));
+      }
     }
   }
   __syncthreads();
-  const int nchosen = min(nsel, kk);
-  uint32_t keys[kMergeItems];
+  // ascending emission: thread t owns words [t * wpt, (t + 1) * wpt)
+  const int wpt = ((words + kMergeThreads - 1) / kMergeThreads + 3) & ~3;
+  const int w_beg = min(words, t * wpt), w_end = min(words, w_beg + wpt);
+  int cnt = 0;
+  for (int w = w_beg; w < w_end; w += 4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(bm + w);
+    cnt += __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
+  }
+  int incl = cnt;
 #pragma unroll
-  for (int e = 0; e < kMergeItems; ++e) {
-    const int i = t * kMergeItems + e;
-    keys[e] = i < nchosen ? chosen[i] : 0xFFFFFFFFu;
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+    if (lane >= d) incl += o;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  const int before = __reduce_add_sync(0xFFFFFFFFu, lane < warp ? wsum[lane] : 0);
+  int pos = before + incl - cnt;
+  int32_t* irow = idx + static_cast<size_t>(u) * p.k;
+  for (int w = w_beg; w < w_end && cnt > 0; ++w) {
+    uint32_t bits = bm[w];
+    while (bits) {
+      const int bpos = __ffs(bits) - 1;
+      bits &= bits - 1u;
+      if (pos < p.k) irow[pos] = 32 * w + bpos;
+      ++pos;
+    }
   }
   __syncthreads();
-  Sort(sm.sort).Sort(keys, 0, kIdxBits);  // indices < 2^21; the pad sorts last (stable)
+  const int chosen_total =
+      min(__reduce_add_sync(0xFFFFFFFFu, wsum[lane]), kk);  // 32 warps: one entry per lane
+  // pad, slots and misses
   int my_miss = 0;
-#pragma unroll
-  for (int e = 0; e < kMergeItems; ++e) {
-    const int j = t * kMergeItems + e;
-    if (j >= p.k) continue;
-    const int i = j < nchosen ? static_cast<int>(keys[e]) : -1;
-    idx[static_cast<size_t>(u) * p.k + j] = i;
+  for (int j = t; j < p.k; j += kMergeThreads) {
+    int i = -1;
+    if (j < chosen_total)
+      i = irow[j];
+    else
+      irow[j] = -1;
     int s = -2;
     if (i >= 0) {
       s = slot_map ? slot_map[static_cast<size_t>(u) * p.n_max + i] : -1;
@@ -497,8 +549,8 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(
     }
     if (slots) slots[static_cast<size_t>(u) * p.k + j] = s;
   }
-  const int w = __reduce_add_sync(0xFFFFFFFFu, my_miss);
-  if ((t & 31) == 0) miss_warp[t >> 5] = w;
+  const int wm = __reduce_add_sync(0xFFFFFFFFu, my_miss);
+  if (lane == 0) miss_warp[warp] = wm;
   __syncthreads();
   if (t == 0 && misses) {
     int m = 0;
@@ -576,7 +628,7 @@ struct FusedLaunch {
 }  // namespace
 
 bool fused_topk_supported(int n_max, int k, int B) {
-  return B > 0 && k >= 1 && k <= kMergeThreads * kMergeItems && 2 * k <= kCandCap - 6144 &&
+  return B > 0 && k >= 1 && k <= kMergeMaxK && 2 * k <= kCandCap - 6144 &&
          n_max <= (1 << kIdxBits);
 }
 
@@ -590,6 +642,7 @@ size_t fused_ws_bytes(int RG, int n_max, int k, int B) {
   c.take<int32_t>(static_cast<size_t>(RG) * L.segs * L.seg_cap);
   c.take<int32_t>(static_cast<size_t>(RG) * L.segs);
   c.take<uint64_t>(static_cast<size_t>(RG) * L.segs * L.seg_cap);
+  c.take<uint32_t>(static_cast<size_t>(RG) * bitmap_words(n_max));
   return c.used;
 }
 
@@ -609,13 +662,14 @@ kvs_status fathom_scan_topk_launch(ScanParams p, void* ws, const int32_t* slot_m
   p.cand_idx = c.take<int32_t>(static_cast<size_t>(p.RG) * L.segs * L.seg_cap);
   p.cand_count = c.take<int32_t>(static_cast<size_t>(p.RG) * L.segs);
   uint64_t* gscratch = c.take<uint64_t>(static_cast<size_t>(p.RG) * L.segs * L.seg_cap);
+  uint32_t* bitmap = c.take<uint32_t>(static_cast<size_t>(p.RG) * bitmap_words(p.n_max));
   kvs_status st = dispatch_schedule(p, FusedLaunch{p, L.grid, s});
   if (st != KVS_OK) return st;
   const size_t msmem = static_cast<size_t>(kMergeSmemEntries) * sizeof(uint64_t);
   cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        static_cast<int>(msmem));
-  topk_merge_kernel<<<p.RG, kMergeThreads, msmem, s>>>(p, L.grid, gscratch, slot_map, idx, slots,
-                                                        misses);
+  topk_merge_kernel<<<p.RG, kMergeThreads, msmem, s>>>(p, L.grid, gscratch, bitmap, slot_map, idx,
+                                                        slots, misses);
   return check_launch("decode_step(top-k merge)");
 }
 
