@@ -9,33 +9,45 @@
 //
 // The rows are read straight from where they live: a staged [k][D] buffer, the
 // hot buffer / full store through the slot of each selected key, or the full
-// store by index. Each block takes a split of one (r, g)'s rows, double-buffers
-// 64-row K/V tiles into shared memory with cp.async (16-byte copies, zero fill
-// for padding rows), computes q.K with one thread per (row, head pair), then a
-// warp per head rescales and accumulates P.V. Splits are merged by their
-// log-sum-exp in a second small kernel. The bound is HBM: 512 bytes of K/V per
-// selected row against ~2 flops per byte.
+// store by index. The bound is the gather of 512 bytes of K/V per row; the
+// arithmetic runs on the tensor cores so that it stays well below it:
+//
+//  * Each warp streams its own 16-row tiles through a three-stage ring in
+//    shared memory with cp.async (16-byte copies, zero fill for padding rows,
+//    chunk c of row r stored at c ^ (r & 7) so that ldmatrix reads are
+//    conflict-free). The row locations of a tile are fetched one tile ahead of
+//    its copies, and its copies two tiles ahead of its arithmetic.
+//  * Logits: S^T[heads][rows] = Q K^T with mma.m16n8k16 (bf16 inputs, f32
+//    accumulation). The 16 MMA rows hold q split in two bf16 parts, q_hi in
+//    rows 0..7 and q - q_hi in rows 8..15, so one MMA carries q to ~16 bits
+//    and the two halves are added in f32.
+//  * P.V: the logit accumulators are, element for element, the A operand of
+//    the next MMA (O[heads][dims] += P[heads][rows] V[rows][dims]); P is split
+//    into hi/lo bf16 parts the same way, V comes from ldmatrix.trans.
+//  * Online softmax per head inside the four lanes that hold it; the block's
+//    warps merge by log-sum-exp in shared memory, and the blocks (splits) of
+//    one (r, g) in a second small kernel.
+#include <cuda_bf16.h>
+
 #include "internal.cuh"
 
 namespace kvs {
 
 namespace {
 
-constexpr int kTile = 64;
-constexpr int kThreads = 128;
-constexpr int kKStride = kD + 8;  // 272-byte K rows in shared memory: conflict-free 16-byte reads
+constexpr int kAttnWarps = 4;
+constexpr int kAttnThreads = 32 * kAttnWarps;
+constexpr int kAttnBlocksPerSM = 2;
+constexpr int kAttnStages = 3;
+constexpr int kTileRows = 16;
+constexpr int kSplitUnit = 64;                           // rows: the granularity of a split
+constexpr int kStageBytes = 2 * kTileRows * kD * 2;      // K and V of one tile, bf16
+constexpr int kAttnSmem = kAttnWarps * kAttnStages * kStageBytes;  // 96 KB
 
-struct AttnSmem {
-  uint16_t K[2][kTile][kKStride];
-  uint16_t V[2][kTile][kD];
-  float q[8][kD];
-  float lg[8][kTile];
-  const uint16_t* kp[2][kTile];
-  const uint16_t* vp[2][kTile];
-};
-
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
-  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(uint32_t s, const void* gmem, bool valid) {
   const int bytes = valid ? 16 : 0;
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(bytes)
                : "memory");
@@ -45,192 +57,279 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// D = A B + D, m16n8k16, bf16 inputs, f32 accumulators.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Two floats as bf16 (round to nearest even), x in the low half.
+__device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(x, y);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+// x = hi + lo with hi = bf16(x) and lo = bf16(x - hi), for a pair.
+__device__ __forceinline__ void split_bf16(float x, float y, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16(x, y);
+  const float hx = __uint_as_float(hi << 16), hy = __uint_as_float(hi & 0xFFFF0000u);
+  lo = pack_bf16(x - hx, y - hy);
+}
 
-// Pointers of row j of (r, g) = u; null when the row is padding.
-__device__ __forceinline__ void resolve_row(const RowSrc& src, int u, int j,
-                                            const uint16_t*& kp, const uint16_t*& vp) {
-  kp = nullptr;
-  vp = nullptr;
-  if (j >= src.k) return;
+// Where row j of (r, g) = u lives, as one code: -1 padding, c >= 0 row c of
+// the staged / full store, c <= -2 hot slot -2 - c.
+__device__ __forceinline__ int row_code(const RowSrc& src, int u, int j) {
+  if (j >= src.k) return -1;
   if (src.mode == kRowsStaged) {
     const int ke = src.k_eff ? src.k_eff[u] : src.k;
-    if (j < ke) {
-      kp = src.K + (static_cast<size_t>(u) * src.k + j) * kD;
-      vp = src.V + (static_cast<size_t>(u) * src.k + j) * kD;
-    }
-    return;
+    return j < ke ? j : -1;
   }
   const int32_t* irow =
       src.idx + (src.idx_shared ? static_cast<size_t>(u / src.G) : static_cast<size_t>(u)) * src.k;
   const int i = irow[j];
-  if (i < 0) return;
+  if (i < 0) return -1;
   if (src.mode == kRowsSlot) {
-    const int s = src.slots ? src.slots[static_cast<size_t>(u) * src.k + j]
-                            : src.slot_map[static_cast<size_t>(u) * src.n_max + i];
-    if (s >= 0) {
-      kp = src.hotK + (static_cast<size_t>(u) * src.S + s) * kD;
-      vp = src.hotV + (static_cast<size_t>(u) * src.S + s) * kD;
-      return;
-    }
+    const int sl = src.slots ? src.slots[static_cast<size_t>(u) * src.k + j]
+                             : src.slot_map[static_cast<size_t>(u) * src.n_max + i];
+    if (sl >= 0) return -2 - sl;
   }
-  kp = src.K + (static_cast<size_t>(u) * src.n_max + i) * kD;
-  vp = src.V + (static_cast<size_t>(u) * src.n_max + i) * kD;
+  return i;
 }
 
 template <int H>
-__global__ void __launch_bounds__(kThreads) sparse_attn_kernel(
+__global__ void __launch_bounds__(kAttnThreads, kAttnBlocksPerSM) sparse_attn_kernel(
     const void* __restrict__ q, int q_bf16, RowSrc src, int nsplit, int rows_per_split,
     float scale_log2, float* __restrict__ out, float* __restrict__ lse,
     float* __restrict__ part) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
+  extern __shared__ __align__(128) unsigned char attn_smem[];
+  const float ninf = -__int_as_float(0x7f800000);
   const int u = blockIdx.x / nsplit;
   const int split = blockIdx.x % nsplit;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, tq = lane & 3;  // MMA fragment row group / thread in group
   const int j_begin = split * rows_per_split;
   const int j_end = min(src.k, j_begin + rows_per_split);
-  const int ntiles = j_end > j_begin ? (j_end - j_begin + kTile - 1) / kTile : 0;
+  const uint32_t ring = smem_u32(attn_smem) + warp * kAttnStages * kStageBytes;
 
-  for (int e = tid; e < H * kD; e += kThreads) {
-    const size_t off = static_cast<size_t>(u) * H * kD + e;
-    const float v = q_bf16 ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(q)[off])
-                           : reinterpret_cast<const float*>(q)[off];
-    sm.q[e / kD][e % kD] = v * scale_log2;
+  // A operand of the logits MMA: row g = q_hi of head g, row g + 8 = q_lo
+  uint32_t qa[8][4];
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int d0 = 16 * ks + 8 * half + 2 * tq;
+      float x = 0.f, y = 0.f;
+      if (g < H) {
+        const size_t off = (static_cast<size_t>(u) * H + g) * kD + d0;
+        if (q_bf16) {
+          const uint16_t* qq = reinterpret_cast<const uint16_t*>(q) + off;
+          x = bf16_bits_to_float(qq[0]);
+          y = bf16_bits_to_float(qq[1]);
+        } else {
+          const float* qq = reinterpret_cast<const float*>(q) + off;
+          x = qq[0];
+          y = qq[1];
+        }
+        x *= scale_log2;
+        y *= scale_log2;
+      }
+      uint32_t hi, lo;
+      split_bf16(x, y, hi, lo);
+      qa[ks][2 * half] = hi;
+      qa[ks][2 * half + 1] = lo;
+    }
   }
 
-  auto load_tile = [&](int t, int buf) {
-    const int j0 = j_begin + t * kTile;
-    if (tid < kTile) {
-      const uint16_t *kp, *vp;
-      resolve_row(src, u, (j0 + tid < j_end) ? j0 + tid : src.k, kp, vp);
-      sm.kp[buf][tid] = kp;
-      sm.vp[buf][tid] = vp;
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int e = tid; e < 2 * kTile * 16; e += kThreads) {
-      const int which = e >> 10, row = (e >> 4) & (kTile - 1), part16 = e & 15;
-      const uint16_t* base = which ? sm.vp[buf][row] : sm.kp[buf][row];
-      void* dst = which ? static_cast<void*>(&sm.V[buf][row][part16 * 8])
-                        : static_cast<void*>(&sm.K[buf][row][part16 * 8]);
-      const void* srcp = base ? static_cast<const void*>(base + part16 * 8) : q;
-      cp_async16(dst, srcp, base != nullptr);
+  // row bases of this (r, g): staged rows are [u][k], full-store rows [u][n_max]
+  const size_t full_rows = src.mode == kRowsStaged ? static_cast<size_t>(src.k)
+                                                   : static_cast<size_t>(src.n_max);
+  const uint16_t* fK = src.K + static_cast<size_t>(u) * full_rows * kD;
+  const uint16_t* fV = src.V + static_cast<size_t>(u) * full_rows * kD;
+  const uint16_t* hK = src.hotK ? src.hotK + static_cast<size_t>(u) * src.S * kD : fK;
+  const uint16_t* hV = src.hotV ? src.hotV + static_cast<size_t>(u) * src.S * kD : fV;
+
+  // this warp's tiles: rows j_begin + 16 * (warp + kAttnWarps * i)
+  const int ntile_all = j_end > j_begin ? (j_end - j_begin + kTileRows - 1) / kTileRows : 0;
+  const int ntiles = ntile_all > warp ? (ntile_all - warp + kAttnWarps - 1) / kAttnWarps : 0;
+  auto tile_row0 = [&](int i) { return j_begin + kTileRows * (warp + kAttnWarps * i); };
+  // lane r < 16 fetches the code of row r of tile i
+  auto fetch_code = [&](int i) -> int {
+    if (i >= ntiles || lane >= kTileRows) return -1;
+    const int j = tile_row0(i) + lane;
+    return j < j_end ? row_code(src, u, j) : -1;
+  };
+  // copies of tile i (codes in lanes 0..15) into stage st; returns its valid-row mask
+  auto issue = [&](int i, int code, int st) -> unsigned {
+    const unsigned vm = __ballot_sync(0xFFFFFFFFu, lane < kTileRows && code != -1) & 0xFFFFu;
+    if (i < ntiles) {
+      const uint32_t sbase = ring + st * kStageBytes;
+      const int ch = lane & 15;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int rc = 2 * e + (lane >> 4);  // row copy: K rows 0..15, then V rows 0..15
+        const int r = rc & 15;
+        const bool isv = rc >= 16;
+        const int c = __shfl_sync(0xFFFFFFFFu, code, r);
+        const uint16_t* base = c >= 0 ? (isv ? fV : fK) : (isv ? hV : hK);
+        const size_t row = static_cast<size_t>(c >= 0 ? c : (c == -1 ? 0 : -2 - c));
+        const uint32_t dst = sbase + (isv ? kTileRows * kD * 2 : 0) + r * (kD * 2) +
+                             ((ch ^ (r & 7)) << 4);
+        cp_async16(dst, base + row * kD + ch * 8, c != -1);
+      }
     }
     cp_async_commit();
+    return vm;
   };
 
-  float m_run[2] = {-__int_as_float(0x7f800000), -__int_as_float(0x7f800000)};
-  float l_run[2] = {0.f, 0.f};
-  float o[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  float o[16][4];
+#pragma unroll
+  for (int d = 0; d < 16; ++d)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[d][e] = 0.f;
+  float m_run = ninf, l_run = 0.f;  // of head g, shared by the four lanes of group g
 
-  if (ntiles > 0) load_tile(0, 0);
-  for (int t = 0; t < ntiles; ++t) {
-    const int buf = t & 1;
-    if (t + 1 < ntiles) {
-      load_tile(t + 1, buf ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
+  // prologue: tiles 0 and 1 in flight, the codes of tile 2 on their way
+  unsigned vm0 = issue(0, fetch_code(0), 0);
+  unsigned vm1 = issue(1, fetch_code(1), 1);
+  int code_next = fetch_code(2);
+
+  for (int i = 0; i < ntiles; ++i) {
+    const int st = i % kAttnStages;
+    const unsigned vm2 = issue(i + 2, code_next, (i + 2) % kAttnStages);
+    code_next = fetch_code(i + 3);
+    cp_async_wait<kAttnStages - 1>();
+    __syncwarp();
+    const uint32_t kst = ring + st * kStageBytes;
+    const uint32_t vst = kst + kTileRows * kD * 2;
+
+    // ---- logits of the tile's 16 rows (two n-tiles of 8) ----
+    float sc[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t b[4];
+      const int row = (lane & 7) + ((lane >> 4) << 3);
+      const int chunk = 2 * ks + ((lane >> 3) & 1);
+      ldsm_x4(kst + row * (kD * 2) + ((chunk ^ (row & 7)) << 4), b);
+      mma_bf16(sc[0], qa[ks], b[0], b[1]);
+      mma_bf16(sc[1], qa[ks], b[2], b[3]);
     }
-    __syncthreads();
-    // ---- logits: thread = (row, head parity) ----
-    {
-      const int row = tid & (kTile - 1), hpar = tid >> 6;
-      constexpr int NH = (H + 1) / 2;
-      float acc[NH];
+    // ---- online softmax of head g over rows n = 8 nt + 2 tq + e ----
+    float s[2][2];
+    float mx = ninf;
 #pragma unroll
-      for (int a = 0; a < NH; ++a) acc[a] = 0.f;
-#pragma unroll 4
-      for (int d8 = 0; d8 < kD / 8; ++d8) {
-        const uint4 kk = *reinterpret_cast<const uint4*>(&sm.K[buf][row][d8 * 8]);
-        const float kf[8] = {__uint_as_float(kk.x << 16), __uint_as_float(kk.x & 0xFFFF0000u),
-                             __uint_as_float(kk.y << 16), __uint_as_float(kk.y & 0xFFFF0000u),
-                             __uint_as_float(kk.z << 16), __uint_as_float(kk.z & 0xFFFF0000u),
-                             __uint_as_float(kk.w << 16), __uint_as_float(kk.w & 0xFFFF0000u)};
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int a = 0; a < NH; ++a) {
-          const int h = hpar + 2 * a;
-          if (h < H) {
-            const float4 q0 = *reinterpret_cast<const float4*>(&sm.q[h][d8 * 8]);
-            const float4 q1 = *reinterpret_cast<const float4*>(&sm.q[h][d8 * 8 + 4]);
-            acc[a] = fmaf(q0.x, kf[0], acc[a]);
-            acc[a] = fmaf(q0.y, kf[1], acc[a]);
-            acc[a] = fmaf(q0.z, kf[2], acc[a]);
-            acc[a] = fmaf(q0.w, kf[3], acc[a]);
-            acc[a] = fmaf(q1.x, kf[4], acc[a]);
-            acc[a] = fmaf(q1.y, kf[5], acc[a]);
-            acc[a] = fmaf(q1.z, kf[6], acc[a]);
-            acc[a] = fmaf(q1.w, kf[7], acc[a]);
-          }
-        }
+      for (int e = 0; e < 2; ++e) {
+        const int n = 8 * nt + 2 * tq + e;
+        const float v = sc[nt][e] + sc[nt][e + 2];
+        s[nt][e] = ((vm0 >> n) & 1u) ? v : ninf;
+        mx = fmaxf(mx, s[nt][e]);
       }
-      const bool valid = sm.kp[buf][row] != nullptr;
+    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    const bool none = m_new == ninf;
+    const float alpha = none ? 1.f : exp2f(m_run - m_new);
+    float p[2][2];
+    float ps = 0.f;
 #pragma unroll
-      for (int a = 0; a < NH; ++a) {
-        const int h = hpar + 2 * a;
-        if (h < H) sm.lg[h][row] = valid ? acc[a] : -__int_as_float(0x7f800000);
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        p[nt][e] = none ? 0.f : exp2f(s[nt][e] - m_new);
+        ps += p[nt][e];
       }
+    ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 1);
+    ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 2);
+    l_run = l_run * alpha + ps;
+    m_run = m_new;
+    if (!__all_sync(0xFFFFFFFFu, alpha == 1.f)) {
+#pragma unroll
+      for (int d = 0; d < 16; ++d)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[d][e] *= alpha;
     }
-    __syncthreads();
-    // ---- online softmax and P.V: warp w owns heads w and w + 4 ----
+    // ---- P.V: P (hi/lo split) is the A operand, V from ldmatrix.trans ----
+    uint32_t pa[4];
+    split_bf16(p[0][0], p[0][1], pa[0], pa[1]);
+    split_bf16(p[1][0], p[1][1], pa[2], pa[3]);
 #pragma unroll
-    for (int a = 0; a < 2; ++a) {
-      const int h = warp + 4 * a;
-      if (h < H) {
-        const float l0 = sm.lg[h][lane], l1 = sm.lg[h][lane + 32];
-        float mx = fmaxf(l0, l1);
-#pragma unroll
-        for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, d));
-        const float m_new = fmaxf(m_run[a], mx);
-        float alpha = 1.f, p0 = 0.f, p1 = 0.f;
-        if (m_new != -__int_as_float(0x7f800000)) {
-          alpha = exp2f(m_run[a] - m_new);
-          p0 = exp2f(l0 - m_new);
-          p1 = exp2f(l1 - m_new);
-        }
-        float ps = p0 + p1;
-#pragma unroll
-        for (int d = 16; d > 0; d >>= 1) ps += __shfl_xor_sync(0xFFFFFFFFu, ps, d);
-        l_run[a] = l_run[a] * alpha + ps;
-        m_run[a] = m_new;
-        sm.lg[h][lane] = p0;
-        sm.lg[h][lane + 32] = p1;
-        __syncwarp();
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[a][e] *= alpha;
-#pragma unroll 8
-        for (int j = 0; j < kTile; ++j) {
-          const float p = sm.lg[h][j];
-          const uint2 vv = *reinterpret_cast<const uint2*>(&sm.V[buf][j][4 * lane]);
-          o[a][0] = fmaf(p, __uint_as_float(vv.x << 16), o[a][0]);
-          o[a][1] = fmaf(p, __uint_as_float(vv.x & 0xFFFF0000u), o[a][1]);
-          o[a][2] = fmaf(p, __uint_as_float(vv.y << 16), o[a][2]);
-          o[a][3] = fmaf(p, __uint_as_float(vv.y & 0xFFFF0000u), o[a][3]);
-        }
-      }
+    for (int d2 = 0; d2 < 8; ++d2) {
+      uint32_t b[4];
+      const int mi = lane >> 3;
+      const int row = (lane & 7) + 8 * (mi & 1);
+      const int chunk = 2 * d2 + (mi >> 1);
+      ldsm_x4_trans(vst + row * (kD * 2) + ((chunk ^ (row & 7)) << 4), b);
+      mma_bf16(o[2 * d2], pa, b[0], b[1]);
+      mma_bf16(o[2 * d2 + 1], pa, b[2], b[3]);
     }
-    __syncthreads();
+    __syncwarp();  // the stage is refilled by the next iteration's copies
+    vm0 = vm1;
+    vm1 = vm2;
   }
+  cp_async_wait<0>();
+  __syncthreads();
 
-  // ---- write: final output (one split) or a partial (m, l, o) ----
+  // ---- merge the block's warps by log-sum-exp (the ring is free now) ----
+  float* sm_o = reinterpret_cast<float*>(attn_smem);  // [warps][H][kD]
+  float* sm_ml = sm_o + kAttnWarps * H * kD;          // [warps][H][2]
+  if (g < H) {
+    float* dst = sm_o + (warp * H + g) * kD + 2 * tq;
 #pragma unroll
-  for (int a = 0; a < 2; ++a) {
-    const int h = warp + 4 * a;
-    if (h >= H) continue;
+    for (int d = 0; d < 16; ++d)
+      *reinterpret_cast<float2*>(dst + 8 * d) = make_float2(o[d][0] + o[d][2], o[d][1] + o[d][3]);
+    if (tq == 0) {
+      sm_ml[(warp * H + g) * 2] = m_run;
+      sm_ml[(warp * H + g) * 2 + 1] = l_run;
+    }
+  }
+  __syncthreads();
+  for (int h = warp; h < H; h += kAttnWarps) {
+    float M = ninf;
+#pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, sm_ml[(w * H + h) * 2]);
+    float L = 0.f;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (M != ninf) {
+#pragma unroll
+      for (int w = 0; w < kAttnWarps; ++w) {
+        const float sw = exp2f(sm_ml[(w * H + h) * 2] - M);
+        L = fmaf(sm_ml[(w * H + h) * 2 + 1], sw, L);
+        const float4 ow = *reinterpret_cast<const float4*>(sm_o + (w * H + h) * kD + 4 * lane);
+        acc[0] = fmaf(ow.x, sw, acc[0]);
+        acc[1] = fmaf(ow.y, sw, acc[1]);
+        acc[2] = fmaf(ow.z, sw, acc[2]);
+        acc[3] = fmaf(ow.w, sw, acc[3]);
+      }
+    }
     if (nsplit == 1) {
-      const float inv = l_run[a] > 0.f ? 1.f / l_run[a] : 0.f;
-      float4 r4 = make_float4(o[a][0] * inv, o[a][1] * inv, o[a][2] * inv, o[a][3] * inv);
-      *reinterpret_cast<float4*>(out + (static_cast<size_t>(u) * H + h) * kD + 4 * lane) = r4;
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      *reinterpret_cast<float4*>(out + (static_cast<size_t>(u) * H + h) * kD + 4 * lane) =
+          make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
       if (lse && lane == 0)
-        lse[static_cast<size_t>(u) * H + h] =
-            l_run[a] > 0.f ? (m_run[a] + log2f(l_run[a])) * 0.6931471805599453f
-                           : -__int_as_float(0x7f800000);
+        lse[static_cast<size_t>(u) * H + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : ninf;
     } else {
       float* pp = part + ((static_cast<size_t>(u) * nsplit + split) * H + h) * (kD + 4);
-      *reinterpret_cast<float4*>(pp + 4 + 4 * lane) = make_float4(o[a][0], o[a][1], o[a][2], o[a][3]);
+      *reinterpret_cast<float4*>(pp + 4 + 4 * lane) = make_float4(acc[0], acc[1], acc[2], acc[3]);
       if (lane == 0) {
-        pp[0] = m_run[a];
-        pp[1] = l_run[a];
+        pp[0] = M;
+        pp[1] = L;
       }
     }
   }
@@ -270,25 +369,37 @@ __global__ void attn_combine_kernel(const float* __restrict__ part, int nsplit, 
 template <int H>
 kvs_status launch_h(const void* q, int q_bf16, const RowSrc& src, int RG, int nsplit, int rps,
                     float scale_log2, float* out, float* lse, float* part, cudaStream_t s) {
-  const size_t smem = sizeof(AttnSmem);
   cudaFuncSetAttribute(sparse_attn_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       static_cast<int>(smem));
-  sparse_attn_kernel<H><<<RG * nsplit, kThreads, smem, s>>>(q, q_bf16, src, nsplit, rps,
-                                                            scale_log2, out, lse, part);
+                       kAttnSmem);
+  sparse_attn_kernel<H><<<RG * nsplit, kAttnThreads, kAttnSmem, s>>>(q, q_bf16, src, nsplit, rps,
+                                                                     scale_log2, out, lse, part);
   if (nsplit > 1) attn_combine_kernel<<<RG, H * 32, 0, s>>>(part, nsplit, H, out, lse);
   return check_launch("sparse_decode_attn");
 }
 
 }  // namespace
 
-// Split of the k rows across blocks: enough blocks to fill the GPU a few times.
+// Split of the k rows across blocks: the split count that minimises (waves of
+// blocks) x (64-row units per block + one unit of per-block overhead), ties to
+// fewer splits.
 void attn_split(int RG, int k, int& nsplit, int& rows_per_split) {
-  const int tiles = max(1, (k + kTile - 1) / kTile);
-  const int target = 4 * sm_count();
-  nsplit = min(tiles, max(1, (target + RG - 1) / RG));
-  const int tiles_per = (tiles + nsplit - 1) / nsplit;
-  rows_per_split = tiles_per * kTile;
-  nsplit = (tiles + tiles_per - 1) / tiles_per;
+  const int units = max(1, (k + kSplitUnit - 1) / kSplitUnit);
+  const long long slots = static_cast<long long>(kAttnBlocksPerSM) * sm_count();
+  int best = 1;
+  long long best_cost = -1;
+  for (int ns = 1; ns <= min(units, 64); ++ns) {
+    const int per = (units + ns - 1) / ns;
+    const int used = (units + per - 1) / per;
+    const long long waves = (static_cast<long long>(RG) * used + slots - 1) / slots;
+    const long long cost = waves * (per + 1);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = used;
+    }
+  }
+  const int per = (units + best - 1) / best;
+  rows_per_split = per * kSplitUnit;
+  nsplit = (units + per - 1) / per;
 }
 
 size_t attn_ws_bytes(int RG, int H, int k) {
@@ -328,11 +439,13 @@ kvs_status attn_launch(const void* q, int q_bf16, const RowSrc& src, int RG, int
 
 namespace {
 
-// 4 MiB of partial results (R*G*nsplit*H*(128+4) floats). The split count
-// falls as the batch grows (about 4 blocks per SM in all), so the need stays
-// below 8 * SMs * H * 528 bytes: on a 148-SM B200 every size with H <= 4 fits,
-// and only H >= 7 with a few hundred (request, KV head) rows exceeds it.
-// Every GPU that loads this library holds the array until the process exits.
+// 4 MiB of partial results: R*G*nsplit*H*(128+4) floats, none when one split
+// per (r, g) suffices. On a 148-SM B200 at k = 2048 and H = 4 the need is
+// 0.5 MiB up to R*G = 296 (the batches of a decode step) and passes 4 MiB from
+// about R*G = 512 up to 2047, where the rows are cut into several splits;
+// from R*G = 2048 one split suffices and the need is zero. Larger needs are
+// rejected. Every GPU that loads this library holds the array until the
+// process exits.
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 static __device__ __align__(256) float g_attn_scratch[kNoAllocScratchBytes / sizeof(float)];
 

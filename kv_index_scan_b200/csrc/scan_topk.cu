@@ -248,19 +248,27 @@ __global__ void KVS_SCAN_BOUNDS(G, b, W) fathom_scan_topk_kernel(ScanParams p) {
         ix[e] = (i < n && key[e] >= tau) ? ib[i] : 0;
       }
       sync();
+      // one shared-memory atomic per warp and round
+      const int lane = t & 31;
+      const unsigned lt = (1u << lane) - 1u;
+      unsigned m[kRound];
+      int wtot = 0;
 #pragma unroll
       for (int e = 0; e < kRound; ++e) {
-        const int i = base + e * NT + t;
-        const bool take = i < n && key[e] >= tau;
-        const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
-        if (m == 0u) continue;
-        const int lane = t & 31, leader = __ffs(m) - 1;
+        m[e] = __ballot_sync(0xFFFFFFFFu, base + e * NT + t < n && key[e] >= tau);
+        wtot += __popc(m[e]);
+      }
+      if (wtot > 0) {
         int pos = 0;
-        if (lane == leader) pos = atomicAdd(&st->cnt2, __popc(m));
-        pos = __shfl_sync(0xFFFFFFFFu, pos, leader) + __popc(m & ((1u << lane) - 1u));
-        if (take) {
-          kb[pos] = key[e];
-          ib[pos] = ix[e];
+        if (lane == 0) pos = atomicAdd(&st->cnt2, wtot);
+        pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
+#pragma unroll
+        for (int e = 0; e < kRound; ++e) {
+          if ((m[e] >> lane) & 1u) {
+            kb[pos + __popc(m[e] & lt)] = key[e];
+            ib[pos + __popc(m[e] & lt)] = ix[e];
+          }
+          pos += __popc(m[e]);
         }
       }
     }
