@@ -328,6 +328,26 @@ KVS_API kvs_status decode_step(const kvs_decode_args* a, void* ws, size_t ws_byt
 KVS_API size_t kvs_decode_step_workspace_size(int32_t R, int32_t G, int32_t H, int32_t n_max, int32_t k,
                                       int32_t B);
 
+/* decode_step_timed -- decode_step that also records caller-created CUDA
+ * events (cudaEvent_t handles, passed as void*) on `stream` at the boundaries
+ * of its stages, so that a caller can time each stage on the device:
+ *   events[0] before the bit allocation (a1),
+ *   events[1] after it,
+ *   events[2] after the scan (a2; on the fused path, the scan kernel that
+ *             keeps top-k candidates on chip),
+ *   events[3] after the selection (a3: the candidate merge, or the top-k over
+ *             scores, and the slot lookup),
+ *   events[4] after the attention (a5).
+ * With idx_in the skipped stages record their events back to back. Results,
+ * workspace and errors are exactly those of decode_step; n_events must be
+ * KVS_DECODE_STAGES + 1 and no event may be null (KVS_EINVAL). The events are
+ * only recorded, never waited on or destroyed. The pages define no such call;
+ * it exists to measure the path. */
+#define KVS_DECODE_STAGES 4
+KVS_API kvs_status decode_step_timed(const kvs_decode_args* a, void* ws, size_t ws_bytes,
+                                     int32_t* dev_status, void* stream, void* const* events,
+                                     int32_t n_events);
+
 #ifdef __cplusplus
 }
 #endif

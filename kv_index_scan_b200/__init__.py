@@ -90,6 +90,8 @@ def _declare():
     L.decode_step.restype = I32
     L.kvs_decode_step_workspace_size.argtypes = [I32, I32, I32, I32, I32, I32]
     L.kvs_decode_step_workspace_size.restype = SZ
+    L.decode_step_timed.argtypes = [ctypes.POINTER(DecodeArgsC), P, SZ, P, P, ctypes.POINTER(P), I32]
+    L.decode_step_timed.restype = I32
 
 
 _declare()
@@ -391,6 +393,24 @@ class DecodeStep:
         st = _lib.decode_step(ctypes.byref(a), _ptr(self.ws), self.ws.numel(), _ptr(dev_status),
                               _stream(stream))
         _check(st, "decode_step")
+        return self.out if out is None else out
+
+    DECODE_STAGES = ("allocation", "scan", "selection", "attention")
+
+    def timed(self, q, events, idx_in=None, idx_shared: bool = False, stream=None,
+              dev_status=None, out=None):
+        """decode_step_timed: as __call__, recording the 5 torch.cuda.Event(enable_timing=True)
+        objects in `events` at the stage boundaries (see DECODE_STAGES)."""
+        if len(events) != len(self.DECODE_STAGES) + 1:
+            raise ValueError(f"{len(self.DECODE_STAGES) + 1} events needed")
+        s = stream if stream is not None else torch.cuda.current_stream()
+        for e in events:  # make sure each event exists (torch creates it lazily)
+            e.record(s)
+        evs = (P * len(events))(*[e.cuda_event for e in events])
+        a = self.args(q, idx_in, idx_shared, out)
+        st = _lib.decode_step_timed(ctypes.byref(a), _ptr(self.ws), self.ws.numel(),
+                                    _ptr(dev_status), _stream(s), evs, len(events))
+        _check(st, "decode_step_timed")
         return self.out if out is None else out
 
 

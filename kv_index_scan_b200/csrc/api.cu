@@ -223,8 +223,8 @@ size_t kvs_decode_step_workspace_size(int32_t R, int32_t G, int32_t H, int32_t n
   return decode_ws_bytes(R, G, H, n_max, k, B);
 }
 
-kvs_status decode_step(const kvs_decode_args* a, void* ws, size_t ws_bytes, int32_t* dev_status,
-                       void* stream) {
+static kvs_status decode_step_checked(const kvs_decode_args* a, void* ws, size_t ws_bytes,
+                                      int32_t* dev_status, void* stream, cudaEvent_t const* ev) {
   KVS_REQUIRE(a != nullptr, KVS_EINVAL, "decode_step: args is null");
   KVS_REQUIRE(a->q && a->out && a->fullK && a->fullV && a->n, KVS_EINVAL,
               "decode_step: q/out/fullK/fullV/n must be non-null");
@@ -256,8 +256,24 @@ kvs_status decode_step(const kvs_decode_args* a, void* ws, size_t ws_bytes, int3
                                       a->plan ? a->plan->B : 0);
   KVS_REQUIRE(ws && ws_bytes >= need, KVS_EWORKSPACE, "decode_step: workspace %zu < %zu bytes",
               ws_bytes, need);
-  kvs_status st = decode_step_run(a, ws, dev_status, static_cast<cudaStream_t>(stream));
+  kvs_status st = decode_step_run(a, ws, dev_status, static_cast<cudaStream_t>(stream), ev);
   return st == KVS_OK ? ok() : st;
+}
+
+kvs_status decode_step(const kvs_decode_args* a, void* ws, size_t ws_bytes, int32_t* dev_status,
+                       void* stream) {
+  return decode_step_checked(a, ws, ws_bytes, dev_status, stream, nullptr);
+}
+
+kvs_status decode_step_timed(const kvs_decode_args* a, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, void* stream, void* const* events,
+                             int32_t n_events) {
+  KVS_REQUIRE(events != nullptr && n_events == KVS_DECODE_STAGES + 1, KVS_EINVAL,
+              "decode_step_timed: %d events given, %d needed", n_events, KVS_DECODE_STAGES + 1);
+  for (int i = 0; i < n_events; ++i)
+    KVS_REQUIRE(events[i] != nullptr, KVS_EINVAL, "decode_step_timed: event %d is null", i);
+  return decode_step_checked(a, ws, ws_bytes, dev_status, stream,
+                             reinterpret_cast<cudaEvent_t const*>(events));
 }
 
 }  // extern "C"

@@ -49,8 +49,13 @@ size_t decode_ws_bytes(int R, int G, int H, int n_max, int k, int B) {
 }
 
 kvs_status decode_step_run(const kvs_decode_args* a, void* ws, int32_t* dev_status,
-                           cudaStream_t s) {
+                           cudaStream_t s, cudaEvent_t const* ev) {
   const int R = a->ix->R, G = a->ix->G, RG = R * G;
+  // stage boundaries: 0 start, 1 allocation, 2 scan, 3 selection, 4 attention
+  auto mark = [&](int i) {
+    if (ev) cudaEventRecord(ev[i], s);
+  };
+  mark(0);
   WsCarver c(ws);
   int32_t* slots_ws = c.take<int32_t>(static_cast<size_t>(RG) * a->k);
   void* attn_ws = c.take<unsigned char>(attn_ws_bytes(RG, a->H, a->k));
@@ -66,6 +71,7 @@ kvs_status decode_step_run(const kvs_decode_args* a, void* ws, int32_t* dev_stat
                           a->ix->kvar, RG, B, a->plan->t, a->plan->plane_idx, a->plan->plane_w,
                           a->plan->C, s);
     if (st != KVS_OK) return st;
+    mark(1);
     if (!a->ix->host_mapped && fused_topk_supported(a->n_max, a->k, B)) {
       // scan with on-chip top-k candidates, then the per-row merge (which also
       // writes the slots and misses)
@@ -83,22 +89,28 @@ kvs_status decode_step_run(const kvs_decode_args* a, void* ws, int32_t* dev_stat
       scan_schedule(B, p.G, p.b, p.nsets);
       p.dev_status = dev_status;
       p.k = a->k;
-      st = fathom_scan_topk_launch(p, rest, a->slot_map, a->idx, slots, a->misses, s);
+      st = fathom_scan_topk_launch(p, rest, a->slot_map, a->idx, slots, a->misses, s,
+                                   ev ? ev[2] : nullptr);
       if (st != KVS_OK) return st;
       have_slots = true;
     } else {
       float* scores = static_cast<float*>(rest);
       st = fathom_scan_dispatch(a->ix, a->plan, a->n, a->n_max, scores, dev_status, s);
       if (st != KVS_OK) return st;
+      mark(2);
       st = topk_launch(scores, a->n_max, a->n, R, G, a->k, 1, a->idx, nullptr, s);
       if (st != KVS_OK) return st;
     }
     sel = a->idx;
+  } else {
+    mark(1);
+    mark(2);
   }
   if (!have_slots) {
     st = select_slots_launch(sel, shared, G, a->k, a->slot_map, a->n_max, RG, slots, a->misses, s);
     if (st != KVS_OK) return st;
   }
+  mark(3);
   RowSrc src{};
   src.mode = a->slot_map ? kRowsSlot : kRowsDirect;
   src.K = a->fullK;
@@ -113,8 +125,11 @@ kvs_status decode_step_run(const kvs_decode_args* a, void* ws, int32_t* dev_stat
   src.S = a->S;
   src.G = G;
   src.k = a->k;
-  return attn_launch(a->q, a->q_dtype == KVS_BF16, src, RG, a->H, a->scale, a->out, a->lse,
-                     attn_ws, s);
+  st = attn_launch(a->q, a->q_dtype == KVS_BF16, src, RG, a->H, a->scale, a->out, a->lse,
+                   attn_ws, s);
+  if (st != KVS_OK) return st;
+  mark(4);
+  return KVS_OK;
 }
 
 

@@ -40,7 +40,8 @@ kvs_status fathom_scan_lut_launch(const ScanParams& p, cudaStream_t s);
 bool fused_topk_supported(int n_max, int k, int B);
 size_t fused_ws_bytes(int RG, int n_max, int k, int B);
 kvs_status fathom_scan_topk_launch(ScanParams p, void* ws, const int32_t* slot_map, int32_t* idx,
-                                   int32_t* slots, int32_t* misses, cudaStream_t s);
+                                   int32_t* slots, int32_t* misses, cudaStream_t s,
+                                   cudaEvent_t after_scan = nullptr);
 kvs_status fathom_scan_dispatch(const kvs_fathom_index* ix, const kvs_plan* plan,
                                 const int32_t* n, int n_max, float* scores, int32_t* dev_status,
                                 cudaStream_t s);
@@ -63,7 +64,8 @@ kvs_status attn_launch(const void* q, int q_bf16, const RowSrc& src, int RG, int
                        float* out, float* lse, void* ws, cudaStream_t s);
 size_t decode_ws_bytes(int R, int G, int H, int n_max, int k, int B);
 kvs_status decode_step_run(const kvs_decode_args* a, void* ws, int32_t* dev_status,
-                           cudaStream_t s);
+                           cudaStream_t s,
+                           cudaEvent_t const* ev = nullptr);
 
 const char* g_err_text();
 

@@ -655,7 +655,8 @@ size_t fused_ws_bytes(int RG, int n_max, int k, int B) {
 }
 
 kvs_status fathom_scan_topk_launch(ScanParams p, void* ws, const int32_t* slot_map, int32_t* idx,
-                                   int32_t* slots, int32_t* misses, cudaStream_t s) {
+                                   int32_t* slots, int32_t* misses, cudaStream_t s,
+                                   cudaEvent_t after_scan) {
   const Layout L = fused_layout(p.RG, p.n_max, p.k, p.B);
   if (L.grid <= 0) return KVS_OK;
   if (L.segs > 64) return fail(KVS_EUNSUPPORTED, "decode_step: %d segments per row", L.segs);
@@ -673,6 +674,7 @@ kvs_status fathom_scan_topk_launch(ScanParams p, void* ws, const int32_t* slot_m
   uint32_t* bitmap = c.take<uint32_t>(static_cast<size_t>(p.RG) * bitmap_words(p.n_max));
   kvs_status st = dispatch_schedule(p, FusedLaunch{p, L.grid, s});
   if (st != KVS_OK) return st;
+  if (after_scan) cudaEventRecord(after_scan, s);
   const size_t msmem = static_cast<size_t>(kMergeSmemEntries) * sizeof(uint64_t);
   cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        static_cast<int>(msmem));

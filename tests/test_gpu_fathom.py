@@ -300,3 +300,24 @@ def test_host_mapped_index_scan_and_decode(kvs, B):
             tol = fathom_score_tol(qbar, kmin[r, g], kstep[r, g], B)
             assert np.max(np.abs(sc[r, g] - ref["scores"][r, g])) <= tol
             check_selection(step.idx[r, g].cpu().numpy(), ref["idx"][r, g], ref["scores"][r, g], 512)
+
+
+def test_decode_step_timed_matches_and_records_stages(kvs):
+    """decode_step_timed gives the same results as decode_step and records its
+    five stage events in order on the stream."""
+    R, G, n, B, k = 2, 4, 30000, 92, 512
+    K, V, nl = synth.fathom_kv(R, G, D, n, seed=71)
+    q = synth.queries(R, G, 4, D, seed=71).to(DEV)
+    ix = kvs.build_fathom_index(K.to(DEV), nl)
+    step = kvs.DecodeStep(ix, nl, n, 4, B, k, K.to(DEV), V.to(DEV))
+    step(q)
+    torch.cuda.synchronize()
+    out0, idx0 = step.out.clone(), step.idx.clone()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(step.DECODE_STAGES) + 1)]
+    step.timed(q, ev)
+    torch.cuda.synchronize()
+    assert torch.equal(step.out, out0) and torch.equal(step.idx, idx0)
+    times = [ev[i].elapsed_time(ev[i + 1]) for i in range(len(step.DECODE_STAGES))]
+    assert all(t >= 0 for t in times) and times[1] > 0 and times[3] > 0
+    with pytest.raises(ValueError):
+        step.timed(q, ev[:3])
