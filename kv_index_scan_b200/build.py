@@ -1,25 +1,36 @@
-"""Build libkvscan.so in-tree for sm_100a (nvcc, static CUDA runtime)."""
+"""Build libkvscan.so in-tree for sm_100a (nvcc, static CUDA runtime).
+
+Each .cu file is compiled to an object in parallel (objects under _build/),
+then the objects are linked into the shared library.
+"""
 from __future__ import annotations
 
 import glob
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libkvscan.so")
-NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
-              "-Xcompiler", "-fPIC", "-shared", "-Xcompiler", "-fvisibility=hidden"]
+OBJ_DIR = os.path.join(ROOT, "_build", "kvscan")
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+CFLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
+                 "-Xcompiler", "-fvisibility=hidden"]
 
 
 def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")))
 
 
-def deps() -> list[str]:
-    return (sources() + sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh")))
+def headers() -> list[str]:
+    return (sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh")))
             + [os.path.join(ROOT, "include", "kvscan.h")])
+
+
+def deps() -> list[str]:
+    return sources() + headers()
 
 
 def stale() -> bool:
@@ -29,11 +40,35 @@ def stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps())
 
 
+def _obj(src: str) -> str:
+    return os.path.join(OBJ_DIR, os.path.basename(src)[:-3] + ".o")
+
+
+def _compile(src: str, verbose: bool) -> str:
+    obj = _obj(src)
+    hdr_t = max(os.path.getmtime(h) for h in headers())
+    if os.path.exists(obj) and os.path.getmtime(obj) >= max(os.path.getmtime(src), hdr_t):
+        return obj
+    cmd = ["nvcc"] + CFLAGS + ["-I" + os.path.join(ROOT, "include"), "-c", src, "-o", obj + ".tmp"]
+    if verbose:
+        print(" ".join(cmd), file=sys.stderr)
+    subprocess.run(cmd, check=True)
+    os.replace(obj + ".tmp", obj)
+    return obj
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not stale():
         return LIB
-    cmd = (["nvcc"] + NVCC_FLAGS + ["-I" + os.path.join(ROOT, "include"), "-o", LIB + ".tmp"]
-           + sources())
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    srcs = sources()
+    if force:
+        for s in srcs:
+            if os.path.exists(_obj(s)):
+                os.remove(_obj(s))
+    with ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+        objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
+    cmd = ["nvcc"] + ARCH + ["-shared", "-o", LIB + ".tmp"] + objs
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
