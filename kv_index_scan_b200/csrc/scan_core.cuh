@@ -38,6 +38,7 @@ struct ScanParams {
   uint32_t* cand_key;   // [RG][segs][seg_cap] per-segment candidates
   int32_t* cand_idx;
   int32_t* cand_count;  // [RG][segs]
+  uint32_t* cand_tau;   // [RG][segs] score key below which a segment's entries are not needed
 };
 
 // Picks the lookup schedule for a budget of B planes: the fewest groups per

@@ -37,6 +37,7 @@
 // top-k candidates on chip (scan_topk.cu shares this kernel's core).
 #include "internal.cuh"
 #include "scan_core.cuh"
+#include "scan_prmt.cuh"
 
 namespace kvs {
 
@@ -91,9 +92,48 @@ struct LutLaunch {
   }
 };
 
+// Plans of at most 144 planes: the byte-indexed lookup core (scan_prmt.cuh).
+// Thread t writes the 16 consecutive scores of its half plane word.
+__global__ void __launch_bounds__(kPThreads, 1) fathom_scan_prmt_kernel(ScanParams p) {
+  ScanCoreP core(p);
+  core.run([&](int u, int c, int nr, const float (&acc)[kPKeys], int t, unsigned char*) {
+    const int i0 = ScanCoreP::key0(c, t);
+    if (i0 >= p.n_max) return;
+    float* out = p.scores + static_cast<size_t>(u) * p.n_max;
+    const float ninf = -__int_as_float(0x7f800000);
+    if (i0 + kPKeys <= p.n_max && (p.n_max & 3) == 0) {
+#pragma unroll
+      for (int j = 0; j < kPKeys; j += 4) {
+        float4 v;
+        v.x = i0 + j + 0 < nr ? acc[j + 0] : ninf;
+        v.y = i0 + j + 1 < nr ? acc[j + 1] : ninf;
+        v.z = i0 + j + 2 < nr ? acc[j + 2] : ninf;
+        v.w = i0 + j + 3 < nr ? acc[j + 3] : ninf;
+        *reinterpret_cast<float4*>(out + i0 + j) = v;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kPKeys; ++j)
+        if (i0 + j < p.n_max) out[i0 + j] = i0 + j < nr ? acc[j] : ninf;
+    }
+  });
+}
+
 }  // namespace
 
 kvs_status fathom_scan_lut_launch(const ScanParams& p, cudaStream_t s) {
+  if (p.B <= kPMaxB) {
+    ScanParams q = p;
+    q.chunks_per_row = prmt_chunks_per_row(p.n_max);
+    q.nstage = prmt_nstages(p.B, 0);
+    const int chunks = q.RG * q.chunks_per_row;
+    if (chunks <= 0) return KVS_OK;
+    const size_t smem = prmt_smem_bytes(p.B, q.nstage, 0);
+    cudaFuncSetAttribute(fathom_scan_prmt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem));
+    fathom_scan_prmt_kernel<<<min(chunks, sm_count()), kPThreads, smem, s>>>(q);
+    return check_launch("index_scan(fathom, prmt)");
+  }
   return dispatch_schedule(p, LutLaunch{p, s});
 }
 

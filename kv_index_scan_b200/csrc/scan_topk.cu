@@ -24,6 +24,7 @@
 // hot-buffer slot map (slots; misses = the number absent from the hot buffer).
 #include "internal.cuh"
 #include "scan_core.cuh"
+#include "scan_prmt.cuh"
 
 namespace kvs {
 
@@ -32,6 +33,7 @@ namespace {
 constexpr int kIdxBits = 21;
 constexpr uint32_t kIdxMask = (1u << kIdxBits) - 1u;
 constexpr int kCandCap = 16384;  // per-block candidate buffer entries in global memory
+constexpr int kPCandCap = 24576; // per-segment candidates of the byte-indexed fused scan
 
 __device__ __forceinline__ uint64_t make_composite(uint32_t key, int idx) {
   return (static_cast<uint64_t>(key) << kIdxBits) |
@@ -418,6 +420,268 @@ __global__ void KVS_SCAN_BOUNDS(G, b, W) fathom_scan_topk_kernel(ScanParams p) {
   });
 }
 
+// ---------------------------------------------------------------------------
+// Fused scan + top-k on the byte-indexed lookup core (plans of <= 144 planes).
+//
+// Each consumer thread holds 16 scores per chunk. A segment's candidates are
+// appended straight into its output region (capacity kPCandCap): a thread
+// builds a 16-bit mask of its keys at or above the running threshold tau, the
+// warp sums the masks' counts with one shuffle scan and one shared atomic, and
+// the passing keys (read back from the warp's scratch band of the consumed
+// stage slot, so only passing keys are visited) are written as
+// (order-preserving score key, index).
+//
+// tau: the segment's first chunk (when it holds >= k valid keys) is binned
+// linearly over [min, max] of its scores into 2048 bins; tau becomes the
+// smallest score in the bin holding the k-th largest, so exactly the keys of
+// that bin and above are held. Every later appended key is counted in its
+// bin; whenever the held count has grown by k/4 since the last raise, the bin b
+// holding the k-th largest held key is found and tau rises to the lower edge
+// of bin b - 1 (one bin of margin against rounding). A segment of n keys then
+// appends about k (1 + ln(n / 4096)) keys (~9,000 for 113K keys, ~10,500 for
+// 230K), well inside the capacity. So at least k held keys
+// are >= tau at all times and the held set is a superset of the segment's
+// top-k. If the held count nears the capacity (ties, degenerate ranges), the
+// held set is cut to exactly the k best by (score, index) and, since later
+// keys have larger indices, only keys strictly above the k-th score are
+// appended afterwards. The segment's final tau is stored beside its count; the
+// merge drops entries below it.
+struct SegStateP {
+  int cnt, fresh, tau_set, strict, hist_on, next_raise;
+  float tau_f, lo, w, inv_w;
+  float red_min[kPWarps], red_max[kPWarps];
+  SelectState sel;
+};
+
+__device__ __forceinline__ int score_bin(float s, float lo, float inv_w) {
+  return min(2047, max(0, static_cast<int>((s - lo) * inv_w)));
+}
+
+__global__ void __launch_bounds__(kPThreads, 1) fathom_scan_topk_prmt_kernel(ScanParams p) {
+  ScanCoreP core(p);
+  constexpr int NT = ScanCoreP::NCONS;
+  constexpr int CK = 32 * kPChunkWords;  // keys per chunk
+  constexpr int NK = kPKeys;
+  unsigned* hist = reinterpret_cast<unsigned*>(core.extra());
+  SegStateP* st = reinterpret_cast<SegStateP*>(hist + 2048);
+  auto sync = [] { ScanCoreP::sync(); };
+  const long long C = static_cast<long long>(p.RG) * p.chunks_per_row;
+  if (threadIdx.x == 0) {
+    st->cnt = 0;
+    st->fresh = 1;
+    st->tau_set = 0;
+    st->strict = 0;
+    st->hist_on = 0;
+  }
+  // (visible to the consumers through the barrier at the first row change)
+  const float pinf = __int_as_float(0x7f800000), ninf = -pinf;
+  // this block's last chunk, and the current segment (one per row the block touches)
+  const int last_chunk = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * C / gridDim.x) - 1;
+  int seg_u = -1;
+  size_t seg = 0;
+
+  core.run([&](int u, int c, int nr, const float (&acc)[NK], int t, unsigned char* slot) {
+    const int lane = t & 31, warp = t >> 5;
+    const int i0 = ScanCoreP::key0(c, t);
+    const int nv = nr - i0;
+    const uint32_t vmask = nv >= NK ? 0xFFFFu : (nv <= 0 ? 0u : ((1u << nv) - 1u));
+    if (u != seg_u) {
+      const int seg_slot = static_cast<int>(blockIdx.x) -
+                           block_of_chunk(static_cast<long long>(u) * p.chunks_per_row, C, gridDim.x);
+      seg = static_cast<size_t>(u) * p.segs_per_row + seg_slot;
+      seg_u = u;
+    }
+    uint32_t* kb = p.cand_key + seg * p.seg_cap;
+    int32_t* ib = p.cand_idx + seg * p.seg_cap;
+
+    // 0. the segment's first chunk: tau from its own scores (its held keys are
+    // then already counted in the histogram)
+    bool binned_now = false;
+    if (st->fresh) {
+      if (nr - 32 * c * kPChunkWords >= p.k) {
+        float mn = pinf, mx = ninf;
+#pragma unroll
+        for (int j = 0; j < NK; ++j)
+          if ((vmask >> j) & 1u) {
+            mn = fminf(mn, acc[j]);
+            mx = fmaxf(mx, acc[j]);
+          }
+        for (int d = 16; d > 0; d >>= 1) {
+          mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, d));
+          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, d));
+        }
+        if (lane == 0) {
+          st->red_min[warp] = mn;
+          st->red_max[warp] = mx;
+        }
+        for (int b = t; b < 2048; b += NT) hist[b] = 0;
+        sync();
+        float lo = st->red_min[0], hi = st->red_max[0];
+#pragma unroll
+        for (int q = 1; q < kPWarps; ++q) {
+          lo = fminf(lo, st->red_min[q]);
+          hi = fmaxf(hi, st->red_max[q]);
+        }
+        const float w = (hi - lo) * (1.0f / 2048.0f);
+        // bins are usable when one bin is well above the rounding of scores
+        const float mag = fmaxf(fabsf(lo), fabsf(hi));
+        const bool usable = hi > lo && w > 16.0f * mag * 5.96e-8f;
+        if (usable) {
+          const float inv_w = 2048.0f / (hi - lo);
+          binned_now = true;
+#pragma unroll
+          for (int j = 0; j < NK; ++j)
+            if ((vmask >> j) & 1u) atomicAdd(&hist[score_bin(acc[j], lo, inv_w)], 1u);
+          sync();
+          find_bin_from_top(hist, 2048, p.k, st->sel.wsum, st->sel.res, t, NT, sync);
+          const int bstar = st->sel.res[0];
+          // tau = the smallest score in bin bstar (exact: bins are monotone in the score)
+          float bmin = pinf;
+#pragma unroll
+          for (int j = 0; j < NK; ++j)
+            if (((vmask >> j) & 1u) && score_bin(acc[j], lo, inv_w) == bstar) bmin = fminf(bmin, acc[j]);
+          for (int d = 16; d > 0; d >>= 1) bmin = fminf(bmin, __shfl_xor_sync(0xFFFFFFFFu, bmin, d));
+          // the held keys are exactly bins >= bstar: clear the rest of the histogram
+          for (int b = t; b < bstar; b += NT) hist[b] = 0;
+          sync();
+          if (lane == 0) st->red_min[warp] = bmin;
+          sync();
+          if (t == 0) {
+            float tm = st->red_min[0];
+            for (int q = 1; q < kPWarps; ++q) tm = fminf(tm, st->red_min[q]);
+            st->tau_f = tm;
+            st->tau_set = 1;
+            st->hist_on = 1;
+            st->lo = lo;
+            st->w = w;
+            st->inv_w = inv_w;
+            st->next_raise = p.k + max(256, p.k / 4);
+          }
+        }
+      } else {
+        sync();  // every thread has read `fresh` before it is cleared
+      }
+      if (t == 0) st->fresh = 0;
+      sync();
+    }
+
+    // 1. keys at or above tau join the segment's candidates
+    const bool has_tau = st->tau_set != 0, strict = st->strict != 0;
+    const bool count_bins = st->hist_on != 0 && !binned_now;
+    const float tau = st->tau_f;
+    uint32_t mask = 0u;
+#pragma unroll
+    for (int j = 0; j < NK; ++j) {
+      const bool pass = !has_tau || (strict ? acc[j] > tau : acc[j] >= tau);
+      mask |= pass ? (1u << j) : 0u;
+    }
+    mask &= vmask;
+    if (__any_sync(0xFFFFFFFFu, mask != 0u)) {
+      // this warp's scratch: rows 0..31 of its 64-byte column band of the slot
+      // (the band only this warp read); lane L's 16 scores in row L
+      float4* row = reinterpret_cast<float4*>(slot + lane * kPRowBytes + 64 * warp);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        row[(q + lane) & 3] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+      const int cnt = __popc(mask);
+      int incl = cnt;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += o;
+      }
+      int base = 0;
+      if (lane == 31) base = atomicAdd(&st->cnt, incl);
+      base = __shfl_sync(0xFFFFFFFFu, base, 31);
+      int pos = base + incl - cnt;
+      __syncwarp();
+      const float* rowf = reinterpret_cast<const float*>(row);
+      const float lo = st->lo, inv_w = st->inv_w;
+      uint32_t mm = mask;
+      while (mm) {
+        const int j = __ffs(mm) - 1;
+        mm &= mm - 1u;
+        const float sc = rowf[4 * (((j >> 2) + lane) & 3) + (j & 3)];
+        if (pos < p.seg_cap) {
+          kb[pos] = ordered_key(sc);
+          ib[pos] = i0 + j;
+        }
+        ++pos;
+        if (count_bins) atomicAdd(&hist[score_bin(sc, lo, inv_w)], 1u);
+      }
+      // scratch rows that are padding planes (B < 32) must be zero again
+      if (lane >= p.B) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) row[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    sync();
+
+    // 2. raise tau from the held keys' histogram once the held set has grown by k
+    if (st->hist_on && st->cnt >= st->next_raise) {
+      find_bin_from_top(hist, 2048, p.k, st->sel.wsum, st->sel.res, t, NT, sync);
+      if (t == 0) {
+        const int b = st->sel.res[0];
+        if (b >= 1) {
+          const float edge = st->lo + static_cast<float>(b - 1) * st->w;
+          if (edge > st->tau_f) st->tau_f = edge;
+        }
+        st->next_raise = st->cnt + max(256, p.k / 4);
+      }
+      sync();
+    }
+
+    // 3. segment end: publish; or make room when the buffer nears capacity
+    const bool seg_end = c == p.chunks_per_row - 1 || u * p.chunks_per_row + c == last_chunk;
+    if (!seg_end && st->cnt > p.seg_cap - CK) {
+      // exact cut to the k best by (score key, index)
+      const int n = st->cnt;
+      uint64_t* comp = p.cbuf_comp + static_cast<size_t>(blockIdx.x) * p.seg_cap;
+      for (int i = t; i < n; i += NT) comp[i] = make_composite(kb[i], ib[i]);
+      sync();
+      const int kk = min(p.k, n);
+      const uint64_t thr = select_kth_composite(comp, n, kk, hist, &st->sel, t, NT, sync);
+      if (t == 0) st->cnt = 0;
+      sync();
+      for (int b0 = 0; b0 < n; b0 += NT) {
+        const int i = b0 + t;
+        const uint64_t cv = i < n ? comp[i] : 0ull;
+        const bool take = i < n && cv >= thr;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
+        if (m == 0u) continue;
+        const int leader = __ffs(m) - 1;
+        int pos = 0;
+        if (lane == leader) pos = atomicAdd(&st->cnt, __popc(m));
+        pos = __shfl_sync(0xFFFFFFFFu, pos, leader) + __popc(m & ((1u << lane) - 1u));
+        if (take) {
+          kb[pos] = static_cast<uint32_t>(cv >> kIdxBits);
+          ib[pos] = composite_index(cv);
+        }
+      }
+      sync();
+      if (t == 0) {
+        st->tau_f = key_to_float(static_cast<uint32_t>(thr >> kIdxBits));
+        st->tau_set = 1;
+        st->strict = 1;
+        st->hist_on = 0;
+      }
+      sync();
+    }
+    if (seg_end) {
+      if (t == 0) {
+        p.cand_count[seg] = min(st->cnt, p.seg_cap);
+        p.cand_tau[seg] = st->tau_set ? ordered_key(st->tau_f) : 0u;
+        st->cnt = 0;
+        st->fresh = 1;
+        st->tau_set = 0;
+        st->strict = 0;
+        st->hist_on = 0;
+      }
+      sync();
+    }
+  });
+}
+
 // One block per (r, g): gather the segments' candidates, select the k best,
 // emit their indices in ascending order, look up their slots. 1024 threads.
 // The ascending order comes from a bitmap over the row's key indices (in the
@@ -426,7 +690,7 @@ __global__ void KVS_SCAN_BOUNDS(G, b, W) fathom_scan_topk_kernel(ScanParams p) {
 // position, and the threads write the set bits of their runs in order.
 constexpr int kMergeThreads = 1024;
 constexpr int kMergeMaxK = 4096;
-constexpr int kMergeSmemEntries = 20480;
+constexpr int kMergeSmemEntries = 24576;
 static_assert(kMergeThreads == 32 * 32, "the merge sums its per-warp counts with one warp");
 
 __host__ __device__ __forceinline__ int bitmap_words(int n_max) {
@@ -440,6 +704,8 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(
   __shared__ unsigned hist[2048];
   __shared__ SelectState sel;
   __shared__ int seg_count[64], seg_off[65];
+  __shared__ uint32_t seg_tau[64];
+  __shared__ int kept_total;
   __shared__ int wsum[kMergeThreads / 32];
   __shared__ int miss_warp[kMergeThreads / 32];
   extern __shared__ __align__(16) uint64_t comp_smem[];
@@ -452,7 +718,11 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(
   const int b0 = block_of_chunk(static_cast<long long>(u) * p.chunks_per_row, C, scan_grid);
   const int b1 = block_of_chunk(static_cast<long long>(u + 1) * p.chunks_per_row - 1, C, scan_grid);
   const int segs = b1 - b0 + 1;
-  if (t < segs) seg_count[t] = p.cand_count[static_cast<size_t>(u) * p.segs_per_row + t];
+  if (t < segs) {
+    seg_count[t] = p.cand_count[static_cast<size_t>(u) * p.segs_per_row + t];
+    seg_tau[t] = p.cand_tau ? p.cand_tau[static_cast<size_t>(u) * p.segs_per_row + t] : 0u;
+  }
+  if (t == 0) kept_total = 0;
   __syncthreads();
   if (t == 0) {
     int o = 0;
@@ -468,34 +738,63 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(
   for (int w = 4 * t; w < words; w += 4 * kMergeThreads)
     *reinterpret_cast<uint4*>(bm + w) = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
-  const int total = seg_off[segs];
-  uint64_t* comp = total <= kMergeSmemEntries
-                       ? comp_smem
-                       : gscratch + static_cast<size_t>(u) * p.segs_per_row * p.seg_cap;
-  // gather the candidates as composites, four loads in flight per thread
-  for (int base = 0; base < total; base += 4 * kMergeThreads) {
-    uint32_t key[4];
-    int32_t ix[4];
+  const int all = seg_off[segs];
+  // entries below their segment's threshold are not needed; count the rest
+  // first when all of them would not fit in shared memory
+  bool in_smem = all <= kMergeSmemEntries;
+  if (!in_smem) {
+    int mine = 0;
+    for (int f = t; f < all; f += kMergeThreads) {
+      int s = 0;
+      while (f >= seg_off[s + 1]) ++s;
+      const size_t off = (static_cast<size_t>(u) * p.segs_per_row + s) * p.seg_cap + (f - seg_off[s]);
+      mine += p.cand_key[off] >= seg_tau[s] ? 1 : 0;
+    }
+    mine = __reduce_add_sync(0xFFFFFFFFu, mine);
+    if (lane == 0) atomicAdd(&kept_total, mine);
+    __syncthreads();
+    in_smem = kept_total <= kMergeSmemEntries;
+    __syncthreads();
+    if (t == 0) kept_total = 0;
+    __syncthreads();
+  }
+  uint64_t* comp =
+      in_smem ? comp_smem : gscratch + static_cast<size_t>(u) * p.segs_per_row * p.seg_cap;
+  // gather the kept candidates as composites: keys and indices of eight
+  // entries per thread in flight together
+  for (int base = 0; base < all; base += 8 * kMergeThreads) {
+    uint32_t key[8], kt[8];
+    int32_t ix[8];
+    bool keep[8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
+    for (int e = 0; e < 8; ++e) {
       const int f = base + e * kMergeThreads + t;
       key[e] = 0u;
       ix[e] = 0;
-      if (f < total) {
+      kt[e] = 0xFFFFFFFFu;
+      if (f < all) {
         int s = 0;
         while (f >= seg_off[s + 1]) ++s;
         const size_t off = (static_cast<size_t>(u) * p.segs_per_row + s) * p.seg_cap + (f - seg_off[s]);
         key[e] = p.cand_key[off];
         ix[e] = p.cand_idx[off];
+        kt[e] = seg_tau[s];
       }
     }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int f = base + e * kMergeThreads + t;
-      if (f < total) comp[f] = make_composite(key[e], ix[e]);
+    for (int e = 0; e < 8; ++e) keep[e] = base + e * kMergeThreads + t < all && key[e] >= kt[e];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const unsigned m = __ballot_sync(0xFFFFFFFFu, keep[e]);
+      if (m == 0u) continue;
+      int pos = 0;
+      if (lane == 0) pos = atomicAdd(&kept_total, __popc(m));
+      pos = __shfl_sync(0xFFFFFFFFu, pos, 0) + __popc(m & ((1u << lane) - 1u));
+      if (keep[e]) comp[pos] = make_composite(key[e], ix[e]);
     }
   }
   __syncthreads();
+  const int total = kept_total;
   uint64_t tau = 0ull;
   if (kk > 0 && total > kk)
     tau = select_kth_composite(comp, total, kk, hist, &sel, t, kMergeThreads,
@@ -587,16 +886,25 @@ struct Layout {
   int grid, cpr, segs, seg_cap;
 };
 
+// Plans of <= 144 planes run the byte-indexed core, whose segments hold up to
+// kPCandCap candidates each; longer plans the group-table core (2k each).
 Layout fused_layout(int RG, int n_max, int k, int B) {
-  int G, b, nsets;
-  scan_schedule(B, G, b, nsets);
   Layout L{};
-  L.cpr = scan_chunks_per_row(n_max, scan_warps(G, b));
+  if (B <= kPMaxB) {
+    L.cpr = prmt_chunks_per_row(n_max);
+    L.seg_cap = kPCandCap;
+  } else {
+    int G, b, nsets;
+    scan_schedule(B, G, b, nsets);
+    L.cpr = scan_chunks_per_row(n_max, scan_warps(G, b));
+    L.seg_cap = 2 * k;
+  }
   L.grid = fused_grid(RG, L.cpr);
   L.segs = L.grid > 0 ? fused_segs_per_row(RG, L.cpr, L.grid) : 1;
-  L.seg_cap = 2 * k;
   return L;
 }
+
+constexpr size_t kPFusedExtra = 2048 * sizeof(unsigned) + sizeof(SegStateP);
 
 struct FusedLaunch {
   const ScanParams& p;
@@ -643,12 +951,14 @@ bool fused_topk_supported(int n_max, int k, int B) {
 size_t fused_ws_bytes(int RG, int n_max, int k, int B) {
   const Layout L = fused_layout(RG, n_max, k, B);
   WsCarver c(nullptr);
+  const size_t cap = static_cast<size_t>(kCandCap > L.seg_cap ? kCandCap : L.seg_cap);
   c.take<uint32_t>(static_cast<size_t>(L.grid) * kCandCap);
   c.take<int32_t>(static_cast<size_t>(L.grid) * kCandCap);
-  c.take<uint64_t>(static_cast<size_t>(L.grid) * kCandCap);
+  c.take<uint64_t>(static_cast<size_t>(L.grid) * cap);
   c.take<uint32_t>(static_cast<size_t>(RG) * L.segs * L.seg_cap);
   c.take<int32_t>(static_cast<size_t>(RG) * L.segs * L.seg_cap);
   c.take<int32_t>(static_cast<size_t>(RG) * L.segs);
+  c.take<uint32_t>(static_cast<size_t>(RG) * L.segs);
   c.take<uint64_t>(static_cast<size_t>(RG) * L.segs * L.seg_cap);
   c.take<uint32_t>(static_cast<size_t>(RG) * bitmap_words(n_max));
   return c.used;
@@ -664,15 +974,29 @@ kvs_status fathom_scan_topk_launch(ScanParams p, void* ws, const int32_t* slot_m
   p.segs_per_row = L.segs;
   p.seg_cap = L.seg_cap;
   WsCarver c(ws);
+  const size_t cap = static_cast<size_t>(kCandCap > L.seg_cap ? kCandCap : L.seg_cap);
   p.cbuf_key = c.take<uint32_t>(static_cast<size_t>(L.grid) * kCandCap);
   p.cbuf_idx = c.take<int32_t>(static_cast<size_t>(L.grid) * kCandCap);
-  p.cbuf_comp = c.take<uint64_t>(static_cast<size_t>(L.grid) * kCandCap);
+  p.cbuf_comp = c.take<uint64_t>(static_cast<size_t>(L.grid) * cap);
   p.cand_key = c.take<uint32_t>(static_cast<size_t>(p.RG) * L.segs * L.seg_cap);
   p.cand_idx = c.take<int32_t>(static_cast<size_t>(p.RG) * L.segs * L.seg_cap);
   p.cand_count = c.take<int32_t>(static_cast<size_t>(p.RG) * L.segs);
+  p.cand_tau = c.take<uint32_t>(static_cast<size_t>(p.RG) * L.segs);
   uint64_t* gscratch = c.take<uint64_t>(static_cast<size_t>(p.RG) * L.segs * L.seg_cap);
   uint32_t* bitmap = c.take<uint32_t>(static_cast<size_t>(p.RG) * bitmap_words(p.n_max));
-  kvs_status st = dispatch_schedule(p, FusedLaunch{p, L.grid, s});
+  kvs_status st;
+  if (p.B <= kPMaxB) {
+    p.nstage = prmt_nstages(p.B, kPFusedExtra);
+    if (p.nstage < 2) return fail(KVS_EUNSUPPORTED, "decode_step: no room for two stages at B=%d", p.B);
+    const size_t smem = prmt_smem_bytes(p.B, p.nstage, kPFusedExtra);
+    cudaFuncSetAttribute(fathom_scan_topk_prmt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem));
+    fathom_scan_topk_prmt_kernel<<<L.grid, kPThreads, smem, s>>>(p);
+    st = check_launch("decode_step(scan+topk, prmt)");
+  } else {
+    p.cand_tau = nullptr;
+    st = dispatch_schedule(p, FusedLaunch{p, L.grid, s});
+  }
   if (st != KVS_OK) return st;
   if (after_scan) cudaEventRecord(after_scan, s);
   const size_t msmem = static_cast<size_t>(kMergeSmemEntries) * sizeof(uint64_t);

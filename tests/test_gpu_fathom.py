@@ -276,6 +276,22 @@ def test_decode_step_all_scores_tied_takes_first_indices(kvs):
     assert torch.all(step.misses == k)
 
 
+def test_decode_step_all_tied_long_rows_cut_to_first_indices(kvs):
+    """All scores equal on rows long enough that a scan block holds more than
+    four 4096-key chunks of one row: its candidate buffer fills, is cut to the
+    k best by (score, index), and later ties must lose to the held ones; the
+    top-k is still the first k indices of every row."""
+    R, G, H, n, k = 4, 2, 4, 327680, 2048
+    K = torch.full((R, G, n, D), -1.25, dtype=torch.bfloat16)
+    V = torch.zeros((R, G, n, D), dtype=torch.bfloat16)
+    q = synth.queries(R, G, H, D, seed=32)
+    ix = kvs.build_fathom_index(K.to(DEV), [n] * R)
+    step = kvs.DecodeStep(ix, [n] * R, n, H, 92, k, K.to(DEV), V.to(DEV))
+    step(q.to(DEV))
+    torch.cuda.synchronize()
+    assert torch.equal(step.idx.cpu(), torch.arange(k, dtype=torch.int32).expand(R, G, k))
+
+
 @pytest.mark.parametrize("B", [68, 92])
 def test_host_mapped_index_scan_and_decode(kvs, B):
     """The index planes in mapped pinned host memory, read over the host link
