@@ -95,9 +95,9 @@ struct LutLaunch {
 // Plans of at most 144 planes: the byte-indexed lookup core (scan_prmt.cuh).
 // Thread t writes the 16 consecutive scores of its half plane word.
 __global__ void __launch_bounds__(kPThreads, 1) fathom_scan_prmt_kernel(ScanParams p) {
-  ScanCoreP core(p);
+  ScanCoreP<false> core(p);
   core.run([&](int u, int c, int nr, const float (&acc)[kPKeys], int t, unsigned char*) {
-    const int i0 = ScanCoreP::key0(c, t);
+    const int i0 = ScanCoreP<false>::key0(c, t);
     if (i0 >= p.n_max) return;
     float* out = p.scores + static_cast<size_t>(u) * p.n_max;
     const float ninf = -__int_as_float(0x7f800000);

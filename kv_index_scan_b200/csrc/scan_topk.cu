@@ -423,33 +423,36 @@ __global__ void KVS_SCAN_BOUNDS(G, b, W) fathom_scan_topk_kernel(ScanParams p) {
 // ---------------------------------------------------------------------------
 // Fused scan + top-k on the byte-indexed lookup core (plans of <= 144 planes).
 //
-// Each consumer thread holds 16 scores per chunk. A segment's candidates are
-// appended straight into its output region (capacity kPCandCap): a thread
-// builds a 16-bit mask of its keys at or above the running threshold tau, the
-// warp sums the masks' counts with one shuffle scan and one shared atomic, and
-// the passing keys (read back from the warp's scratch band of the consumed
-// stage slot, so only passing keys are visited) are written as
-// (order-preserving score key, index).
+// The eight scoring warps only write each chunk's 4,096 scores into the
+// consumed stage slot (scan_prmt.cuh, staged mode); four selector warps, one
+// per scheduler, read them there (two scoring warps' bands each) and keep the
+// segment's candidates, so the latency of the selection never stalls the
+// scoring warps. A segment's candidates are appended straight into its output
+// region (capacity kPCandCap) as (order-preserving score key, index): a lane
+// marks which of its 32 scores are at or above the running threshold tau, the
+// warp takes its positions with one shuffle scan and one shared atomic, and
+// only the marked scores are read again and written.
 //
 // tau: the segment's first chunk (when it holds >= k valid keys) is binned
 // linearly over [min, max] of its scores into 2048 bins; tau becomes the
 // smallest score in the bin holding the k-th largest, so exactly the keys of
 // that bin and above are held. Every later appended key is counted in its
-// bin; whenever the held count has grown by k/4 since the last raise, the bin b
-// holding the k-th largest held key is found and tau rises to the lower edge
-// of bin b - 1 (one bin of margin against rounding). A segment of n keys then
-// appends about k (1 + ln(n / 4096)) keys (~9,000 for 113K keys, ~10,500 for
-// 230K), well inside the capacity. So at least k held keys
-// are >= tau at all times and the held set is a superset of the segment's
-// top-k. If the held count nears the capacity (ties, degenerate ranges), the
-// held set is cut to exactly the k best by (score, index) and, since later
-// keys have larger indices, only keys strictly above the k-th score are
-// appended afterwards. The segment's final tau is stored beside its count; the
-// merge drops entries below it.
-struct SegStateP {
-  int cnt, fresh, tau_set, strict, hist_on, next_raise;
+// bin. Whenever the held count has grown by k/4 since the last raise, the one
+// selector warp that moves the raise mark (a compare-and-swap) finds the bin b
+// holding the k-th largest held key and raises tau to the lower edge of bin
+// b - 1 (one bin of margin against rounding). The counts it reads may lag
+// appends still in flight, so they are lower bounds: at least k held keys are
+// >= tau at all times and the held set is a superset of the segment's top-k.
+// A segment of n keys appends about k (1 + ln(n / 4096)) keys (~9,000 for
+// 113K keys, ~10,500 for 230K). Every second chunk the selectors check the
+// fill; near capacity (ties, degenerate ranges) the held set is cut to exactly
+// the k best by (score, index) and, since later keys have larger indices, only
+// keys strictly above the k-th score are appended afterwards. The segment's
+// final tau is stored beside its count; the merge drops entries below it.
+struct SelStateP {
+  int cnt, tau_set, strict, hist_on, next_raise;
   float tau_f, lo, w, inv_w;
-  float red_min[kPWarps], red_max[kPWarps];
+  float red_min[kPSel], red_max[kPSel];
   SelectState sel;
 };
 
@@ -457,227 +460,350 @@ __device__ __forceinline__ int score_bin(float s, float lo, float inv_w) {
   return min(2047, max(0, static_cast<int>((s - lo) * inv_w)));
 }
 
-__global__ void __launch_bounds__(kPThreads, 1) fathom_scan_topk_prmt_kernel(ScanParams p) {
-  ScanCoreP core(p);
-  constexpr int NT = ScanCoreP::NCONS;
-  constexpr int CK = 32 * kPChunkWords;  // keys per chunk
-  constexpr int NK = kPKeys;
-  unsigned* hist = reinterpret_cast<unsigned*>(core.extra());
-  SegStateP* st = reinterpret_cast<SegStateP*>(hist + 2048);
-  auto sync = [] { ScanCoreP::sync(); };
-  const long long C = static_cast<long long>(p.RG) * p.chunks_per_row;
-  if (threadIdx.x == 0) {
-    st->cnt = 0;
-    st->fresh = 1;
-    st->tau_set = 0;
-    st->strict = 0;
-    st->hist_on = 0;
+// One warp: the bin holding the k-th largest count of hist (from the top), or
+// -1 when the histogram holds fewer than k. Lane l first sums bins
+// [2048 - 64 (l + 1), 2048 - 64 l) (16-byte reads in a lane-rotated order),
+// then the lane holding the rank is resolved two bins per lane.
+__device__ __forceinline__ int warp_kth_bin(const unsigned* hist, int k, int lane) {
+  const uint4* h4 = reinterpret_cast<const uint4*>(hist);
+  const int q0 = 512 - 16 * (lane + 1);
+  unsigned sum = 0;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const uint4 v = h4[q0 + ((e + lane) & 15)];
+    sum += v.x + v.y + v.z + v.w;
   }
-  // (visible to the consumers through the barrier at the first row change)
-  const float pinf = __int_as_float(0x7f800000), ninf = -pinf;
-  // this block's last chunk, and the current segment (one per row the block touches)
-  const int last_chunk = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * C / gridDim.x) - 1;
-  int seg_u = -1;
-  size_t seg = 0;
+  unsigned incl = sum;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const unsigned o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+    if (lane >= d) incl += o;
+  }
+  const unsigned hit = __ballot_sync(0xFFFFFFFFu, incl >= static_cast<unsigned>(k));
+  if (hit == 0u) return -1;
+  const int L = __ffs(hit) - 1;
+  const unsigned krem = static_cast<unsigned>(k) - __shfl_sync(0xFFFFFFFFu, incl - sum, L);
+  const int b_hi = 2048 - 64 * L - 1 - 2 * lane;
+  const unsigned c_hi = hist[b_hi], c_lo = hist[b_hi - 1];
+  const unsigned c2 = c_hi + c_lo;
+  unsigned incl2 = c2;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const unsigned o = __shfl_up_sync(0xFFFFFFFFu, incl2, d);
+    if (lane >= d) incl2 += o;
+  }
+  const unsigned hit2 = __ballot_sync(0xFFFFFFFFu, incl2 >= krem);
+  const int l2 = hit2 ? __ffs(hit2) - 1 : 31;
+  const unsigned before = __shfl_sync(0xFFFFFFFFu, incl2 - c2, l2);
+  const unsigned top_cnt = __shfl_sync(0xFFFFFFFFu, c_hi, l2);
+  const int bb = 2048 - 64 * L - 1 - 2 * l2;
+  return before + top_cnt >= krem ? bb : bb - 1;
+}
 
-  core.run([&](int u, int c, int nr, const float (&acc)[NK], int t, unsigned char* slot) {
-    const int lane = t & 31, warp = t >> 5;
-    const int i0 = ScanCoreP::key0(c, t);
-    const int nv = nr - i0;
-    const uint32_t vmask = nv >= NK ? 0xFFFFu : (nv <= 0 ? 0u : ((1u << nv) - 1u));
-    if (u != seg_u) {
-      const int seg_slot = static_cast<int>(blockIdx.x) -
-                           block_of_chunk(static_cast<long long>(u) * p.chunks_per_row, C, gridDim.x);
-      seg = static_cast<size_t>(u) * p.segs_per_row + seg_slot;
-      seg_u = u;
-    }
-    uint32_t* kb = p.cand_key + seg * p.seg_cap;
-    int32_t* ib = p.cand_idx + seg * p.seg_cap;
+// Barrier of the selector warps only; and the same returning the OR of a predicate.
+__device__ __forceinline__ void sel_sync() {
+  asm volatile("bar.sync 2, %0;\n" ::"n"(32 * kPSel) : "memory");
+}
+__device__ __forceinline__ bool sel_sync_or(bool pred) {
+  int r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.s32 p, %1, 0;\n bar.red.or.pred q, 2, %2, p;\n"
+      " selp.s32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"(pred ? 1 : 0), "n"(32 * kPSel)
+      : "memory");
+  return r != 0;
+}
 
-    // 0. the segment's first chunk: tau from its own scores (its held keys are
-    // then already counted in the histogram)
-    bool binned_now = false;
-    if (st->fresh) {
-      if (nr - 32 * c * kPChunkWords >= p.k) {
-        float mn = pinf, mx = ninf;
-#pragma unroll
-        for (int j = 0; j < NK; ++j)
-          if ((vmask >> j) & 1u) {
-            mn = fminf(mn, acc[j]);
-            mx = fmaxf(mx, acc[j]);
-          }
-        for (int d = 16; d > 0; d >>= 1) {
-          mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, d));
-          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, d));
+__global__ void __launch_bounds__(kPThreadsStaged, 1) fathom_scan_topk_prmt_kernel(ScanParams p) {
+  using Core = ScanCoreP<true>;
+  Core core(p);
+  unsigned* hist = reinterpret_cast<unsigned*>(core.extra());
+  SelStateP* st = reinterpret_cast<SelStateP*>(hist + 2048);
+  volatile SelStateP* vst = st;
+  core.run([](int, int, int, const float (&)[kPKeys], int, unsigned char*) {}, [&](int beg, int end) {
+    constexpr int NS = 32 * kPSel;
+    constexpr int CK = 32 * kPChunkWords;  // keys per chunk
+    const int lane = threadIdx.x & 31;
+    const int sw = (threadIdx.x >> 5) - (kPWarps + kPProd);
+    const int tid = 32 * sw + lane;
+    const long long C = static_cast<long long>(p.RG) * p.chunks_per_row;
+    const int last_chunk = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * C / gridDim.x) - 1;
+    const int raise_step = max(256, p.k / 4);
+    const float pinf = __int_as_float(0x7f800000), ninf = -pinf;
+    // lane's place in a chunk: iteration e reads row 4e + (lane >> 3), 16 bytes
+    // q4 = lane & 7 of this warp's 128-byte part (scoring warps 2 sw, 2 sw + 1)
+    const int q4 = lane & 7;
+    const int cw = 2 * sw + (q4 >> 2);  // scoring warp whose scores these are
+    int u = beg / p.chunks_per_row, c = beg % p.chunks_per_row, stg = 0;
+    uint32_t phase = 0u;
+    int chunk_i = 0, seg_u = -1;
+    size_t seg = 0;
+    bool fresh = false, dead = false;
+    for (int it = beg; it < end; ++it) {
+      const int nr = p.n[u / p.Gheads];
+      if (u != seg_u) {
+        seg = static_cast<size_t>(u) * p.segs_per_row +
+              (static_cast<int>(blockIdx.x) -
+               block_of_chunk(static_cast<long long>(u) * p.chunks_per_row, C, gridDim.x));
+        seg_u = u;
+        fresh = true;
+        if (tid == 0) {
+          st->cnt = 0;
+          st->tau_set = 0;
+          st->strict = 0;
+          st->hist_on = 0;
         }
-        if (lane == 0) {
-          st->red_min[warp] = mn;
-          st->red_max[warp] = mx;
-        }
-        for (int b = t; b < 2048; b += NT) hist[b] = 0;
-        sync();
-        float lo = st->red_min[0], hi = st->red_max[0];
-#pragma unroll
-        for (int q = 1; q < kPWarps; ++q) {
-          lo = fminf(lo, st->red_min[q]);
-          hi = fmaxf(hi, st->red_max[q]);
-        }
-        const float w = (hi - lo) * (1.0f / 2048.0f);
-        // bins are usable when one bin is well above the rounding of scores
-        const float mag = fmaxf(fabsf(lo), fabsf(hi));
-        const bool usable = hi > lo && w > 16.0f * mag * 5.96e-8f;
-        if (usable) {
-          const float inv_w = 2048.0f / (hi - lo);
-          binned_now = true;
-#pragma unroll
-          for (int j = 0; j < NK; ++j)
-            if ((vmask >> j) & 1u) atomicAdd(&hist[score_bin(acc[j], lo, inv_w)], 1u);
-          sync();
-          find_bin_from_top(hist, 2048, p.k, st->sel.wsum, st->sel.res, t, NT, sync);
-          const int bstar = st->sel.res[0];
-          // tau = the smallest score in bin bstar (exact: bins are monotone in the score)
-          float bmin = pinf;
-#pragma unroll
-          for (int j = 0; j < NK; ++j)
-            if (((vmask >> j) & 1u) && score_bin(acc[j], lo, inv_w) == bstar) bmin = fminf(bmin, acc[j]);
-          for (int d = 16; d > 0; d >>= 1) bmin = fminf(bmin, __shfl_xor_sync(0xFFFFFFFFu, bmin, d));
-          // the held keys are exactly bins >= bstar: clear the rest of the histogram
-          for (int b = t; b < bstar; b += NT) hist[b] = 0;
-          sync();
-          if (lane == 0) st->red_min[warp] = bmin;
-          sync();
-          if (t == 0) {
-            float tm = st->red_min[0];
-            for (int q = 1; q < kPWarps; ++q) tm = fminf(tm, st->red_min[q]);
-            st->tau_f = tm;
-            st->tau_set = 1;
-            st->hist_on = 1;
-            st->lo = lo;
-            st->w = w;
-            st->inv_w = inv_w;
-            st->next_raise = p.k + max(256, p.k / 4);
-          }
-        }
-      } else {
-        sync();  // every thread has read `fresh` before it is cleared
+        sel_sync();
       }
-      if (t == 0) st->fresh = 0;
-      sync();
-    }
-
-    // 1. keys at or above tau join the segment's candidates
-    const bool has_tau = st->tau_set != 0, strict = st->strict != 0;
-    const bool count_bins = st->hist_on != 0 && !binned_now;
-    const float tau = st->tau_f;
-    uint32_t mask = 0u;
-#pragma unroll
-    for (int j = 0; j < NK; ++j) {
-      const bool pass = !has_tau || (strict ? acc[j] > tau : acc[j] >= tau);
-      mask |= pass ? (1u << j) : 0u;
-    }
-    mask &= vmask;
-    if (__any_sync(0xFFFFFFFFu, mask != 0u)) {
-      // this warp's scratch: rows 0..31 of its 64-byte column band of the slot
-      // (the band only this warp read); lane L's 16 scores in row L
-      float4* row = reinterpret_cast<float4*>(slot + lane * kPRowBytes + 64 * warp);
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        row[(q + lane) & 3] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
-      const int cnt = __popc(mask);
-      int incl = cnt;
-#pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= d) incl += o;
+      if (!dead && !mbar_wait(&core.scored[stg], phase)) {
+        core.fail_timeout();
+        dead = true;
       }
-      int base = 0;
-      if (lane == 31) base = atomicAdd(&st->cnt, incl);
-      base = __shfl_sync(0xFFFFFFFFu, base, 31);
-      int pos = base + incl - cnt;
+      unsigned char* slot = g_scan_smem + core.stage0 + stg * core.slot_bytes;
+      uint32_t* kb = p.cand_key + seg * p.seg_cap;
+      int32_t* ib = p.cand_idx + seg * p.seg_cap;
+      // this lane's 32 scores and their validity; score j is key
+      // kbase0 + 64 (j >> 2) + (j & 3)
+      const int kbase0 = 32 * (c * kPChunkWords + 16 * cw + (lane >> 4)) + 16 * ((lane >> 3) & 1) + 4 * (q4 & 3);
+      float4 v[8];
+      uint32_t valid = 0u;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int r = 4 * e + (lane >> 3);
+        v[e] = *reinterpret_cast<const float4*>(slot + r * kPRowBytes + 128 * sw + 16 * q4);
+        const int nv = nr - (kbase0 + 64 * e);
+        valid |= (nv >= 4 ? 15u : (nv <= 0 ? 0u : ((1u << nv) - 1u))) << (4 * e);
+      }
+      auto score = [&](int j) -> float {
+        const float4 f = v[j >> 2];
+        const int cc = j & 3;
+        return cc == 0 ? f.x : (cc == 1 ? f.y : (cc == 2 ? f.z : f.w));
+      };
+      // 0. the segment's first chunk: tau from its own scores (its held keys are
+      // then already counted in the histogram)
+      bool binned_now = false;
+      if (fresh) {
+        fresh = false;
+        if (nr - 32 * c * kPChunkWords >= p.k) {
+          float mn = pinf, mx = ninf;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if ((valid >> j) & 1u) {
+              mn = fminf(mn, score(j));
+              mx = fmaxf(mx, score(j));
+            }
+          for (int d = 16; d > 0; d >>= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, d));
+            mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, d));
+          }
+          if (lane == 0) {
+            st->red_min[sw] = mn;
+            st->red_max[sw] = mx;
+          }
+          for (int b = tid; b < 2048; b += NS) hist[b] = 0;
+          sel_sync();
+          float lo = st->red_min[0], hi = st->red_max[0];
+#pragma unroll
+          for (int q = 1; q < kPSel; ++q) {
+            lo = fminf(lo, st->red_min[q]);
+            hi = fmaxf(hi, st->red_max[q]);
+          }
+          const float w = (hi - lo) * (1.0f / 2048.0f);
+          const float mag = fmaxf(fabsf(lo), fabsf(hi));
+          // bins are usable when one bin is well above the rounding of scores
+          if (hi > lo && w > 16.0f * mag * 5.96e-8f) {  // the same in every selector thread
+            const float inv_w = 2048.0f / (hi - lo);
+            binned_now = true;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if ((valid >> j) & 1u) atomicAdd(&hist[score_bin(score(j), lo, inv_w)], 1u);
+            sel_sync();
+            const int bstar = warp_kth_bin(hist, p.k, lane);  // the same in every warp
+            // tau = the smallest score in bin bstar (exact: bins are monotone in the score)
+            float bmin = pinf;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (((valid >> j) & 1u) && score_bin(score(j), lo, inv_w) == bstar) bmin = fminf(bmin, score(j));
+            for (int d = 16; d > 0; d >>= 1) bmin = fminf(bmin, __shfl_xor_sync(0xFFFFFFFFu, bmin, d));
+            sel_sync();  // every warp has read the histogram
+            // the held keys are exactly bins >= bstar: clear the rest of the histogram
+            for (int b = tid; b < bstar; b += NS) hist[b] = 0;
+            if (lane == 0) st->red_min[sw] = bmin;
+            sel_sync();
+            if (tid == 0) {
+              float tm = st->red_min[0];
+              for (int q = 1; q < kPSel; ++q) tm = fminf(tm, st->red_min[q]);
+              st->tau_f = tm;
+              st->tau_set = 1;
+              st->hist_on = 1;
+              st->lo = lo;
+              st->w = w;
+              st->inv_w = inv_w;
+              st->next_raise = p.k + raise_step;
+            }
+            sel_sync();
+          }
+        }
+      }
+
+      // 1. keys at or above tau join the segment's candidates
+      const bool count_bins = vst->hist_on != 0 && !binned_now;
+      float tau = ninf;
+      if (vst->tau_set) {
+        tau = vst->tau_f;
+        if (vst->strict) tau = nextafterf(tau, pinf);  // strictly above the cut's k-th score
+      }
+      uint32_t mask = 0u;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) mask |= score(j) >= tau ? (1u << j) : 0u;
+      mask &= valid;
+      // appends, in two halves of 16 keys per lane: lane L first writes its
+      // passing (score, key) pairs densely into row L of this warp's part of
+      // the slot (128 bytes: 16 pairs; its scores are in registers now), then
+      // the warp writes them out one pair per lane (each lane finds the pair's
+      // source lane by binary search over the lanes' offsets), with one shared
+      // atomic per half for their positions
       __syncwarp();
-      const float* rowf = reinterpret_cast<const float*>(row);
-      const float lo = st->lo, inv_w = st->inv_w;
-      uint32_t mm = mask;
-      while (mm) {
-        const int j = __ffs(mm) - 1;
-        mm &= mm - 1u;
-        const float sc = rowf[4 * (((j >> 2) + lane) & 3) + (j & 3)];
-        if (pos < p.seg_cap) {
-          kb[pos] = ordered_key(sc);
-          ib[pos] = i0 + j;
-        }
-        ++pos;
-        if (count_bins) atomicAdd(&hist[score_bin(sc, lo, inv_w)], 1u);
-      }
-      // scratch rows that are padding planes (B < 32) must be zero again
-      if (lane >= p.B) {
+      int new_cnt = -1;
+      unsigned char* mine = slot + lane * kPRowBytes + 128 * sw;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) row[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    }
-    sync();
-
-    // 2. raise tau from the held keys' histogram once the held set has grown by k
-    if (st->hist_on && st->cnt >= st->next_raise) {
-      find_bin_from_top(hist, 2048, p.k, st->sel.wsum, st->sel.res, t, NT, sync);
-      if (t == 0) {
-        const int b = st->sel.res[0];
-        if (b >= 1) {
-          const float edge = st->lo + static_cast<float>(b - 1) * st->w;
-          if (edge > st->tau_f) st->tau_f = edge;
+      for (int half = 0; half < 2; ++half) {
+        const uint32_t hm = (mask >> (16 * half)) & 0xFFFFu;
+        const int cnt = __popc(hm);
+        int incl = cnt;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+          const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+          if (lane >= d) incl += o;
         }
-        st->next_raise = st->cnt + max(256, p.k / 4);
+        const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        if (total == 0) continue;
+        uint32_t woff = 0u;
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          const int j = 16 * half + jj;
+          if ((hm >> jj) & 1u) {
+            *reinterpret_cast<uint2*>(mine + woff) = make_uint2(
+                __float_as_uint(score(j)), static_cast<uint32_t>(kbase0 + 64 * (j >> 2) + (j & 3)));
+            woff += 8u;
+          }
+        }
+        int base = 0;
+        if (lane == 0) base = atomicAdd(&st->cnt, total);
+        base = __shfl_sync(0xFFFFFFFFu, base, 0);
+        new_cnt = base + total;
+        const int excl = incl - cnt;
+        __syncwarp();
+        const float lo = st->lo, inv_w = st->inv_w;
+        for (int f0 = 0; f0 < total; f0 += 32) {
+          const int f = f0 + lane;
+          // source lane: the last lane whose exclusive offset is <= f
+          int src = 0;
+#pragma unroll
+          for (int step = 16; step > 0; step >>= 1) {
+            const int probe = src + step;
+            if (__shfl_sync(0xFFFFFFFFu, excl, probe) <= f) src = probe;
+          }
+          const int rank = f - __shfl_sync(0xFFFFFFFFu, excl, src);
+          if (f < total) {
+            const uint2 e = *reinterpret_cast<const uint2*>(slot + src * kPRowBytes + 128 * sw + 8 * rank);
+            const float sc = __uint_as_float(e.x);
+            if (base + f < p.seg_cap) {
+              kb[base + f] = ordered_key(sc);
+              ib[base + f] = static_cast<int32_t>(e.y);
+            }
+            if (count_bins) atomicAdd(&hist[score_bin(sc, lo, inv_w)], 1u);
+          }
+        }
+        __syncwarp();
       }
-      sync();
-    }
-
-    // 3. segment end: publish; or make room when the buffer nears capacity
-    const bool seg_end = c == p.chunks_per_row - 1 || u * p.chunks_per_row + c == last_chunk;
-    if (!seg_end && st->cnt > p.seg_cap - CK) {
-      // exact cut to the k best by (score key, index)
-      const int n = st->cnt;
-      uint64_t* comp = p.cbuf_comp + static_cast<size_t>(blockIdx.x) * p.seg_cap;
-      for (int i = t; i < n; i += NT) comp[i] = make_composite(kb[i], ib[i]);
-      sync();
-      const int kk = min(p.k, n);
-      const uint64_t thr = select_kth_composite(comp, n, kk, hist, &st->sel, t, NT, sync);
-      if (t == 0) st->cnt = 0;
-      sync();
-      for (int b0 = 0; b0 < n; b0 += NT) {
-        const int i = b0 + t;
-        const uint64_t cv = i < n ? comp[i] : 0ull;
-        const bool take = i < n && cv >= thr;
-        const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
-        if (m == 0u) continue;
-        const int leader = __ffs(m) - 1;
-        int pos = 0;
-        if (lane == leader) pos = atomicAdd(&st->cnt, __popc(m));
-        pos = __shfl_sync(0xFFFFFFFFu, pos, leader) + __popc(m & ((1u << lane) - 1u));
-        if (take) {
-          kb[pos] = static_cast<uint32_t>(cv >> kIdxBits);
-          ib[pos] = composite_index(cv);
+      // the warp that moves the raise mark raises tau from the histogram
+      if (count_bins && new_cnt >= 0) {
+        int won = 0;
+        if (lane == 0) {
+          const int mark = vst->next_raise;
+          won = new_cnt >= mark && atomicCAS(&st->next_raise, mark, new_cnt + raise_step) == mark;
+        }
+        if (__shfl_sync(0xFFFFFFFFu, won, 0)) {
+          const int b = warp_kth_bin(hist, p.k, lane);
+          if (lane == 0 && b >= 1) {
+            const float edge = st->lo + static_cast<float>(b - 1) * st->w;
+            if (edge > vst->tau_f) vst->tau_f = edge;
+          }
         }
       }
-      sync();
-      if (t == 0) {
-        st->tau_f = key_to_float(static_cast<uint32_t>(thr >> kIdxBits));
-        st->tau_set = 1;
-        st->strict = 1;
-        st->hist_on = 0;
+
+      // the slot goes back to the producers; rows that are padding planes
+      // (B < 32) must be zero again
+      if (p.B < 32) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (4 * e + (lane >> 3) >= p.B)
+            *reinterpret_cast<float4*>(slot + (4 * e + (lane >> 3)) * kPRowBytes + 128 * sw + 16 * q4) =
+                make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      sync();
-    }
-    if (seg_end) {
-      if (t == 0) {
-        p.cand_count[seg] = min(st->cnt, p.seg_cap);
-        p.cand_tau[seg] = st->tau_set ? ordered_key(st->tau_f) : 0u;
-        st->cnt = 0;
-        st->fresh = 1;
-        st->tau_set = 0;
-        st->strict = 0;
-        st->hist_on = 0;
+      __syncwarp();
+      if (!dead && lane == 0) mbar_arrive(&core.empty[stg]);
+
+      // 3. at the segment's end (publish), and every second chunk (the buffer
+      // may take two more chunks of appends before it must be cut)
+      const bool seg_end = c == p.chunks_per_row - 1 || u * p.chunks_per_row + c == last_chunk;
+      if (seg_end || (chunk_i & 1)) {
+        sel_sync();  // every warp's appends of this chunk are done
+        // one decision for all: the count is read after the barrier, and no warp
+        // appends again before every thread has read it
+        if (sel_sync_or(!seg_end && st->cnt > p.seg_cap - 2 * CK)) {
+          // exact cut to the k best by (score key, index)
+          const int n = st->cnt;
+          uint64_t* comp = p.cbuf_comp + static_cast<size_t>(blockIdx.x) * p.seg_cap;
+          for (int i = tid; i < n; i += NS) comp[i] = make_composite(kb[i], ib[i]);
+          sel_sync();
+          const int kk = min(p.k, n);
+          const uint64_t thr = select_kth_composite(comp, n, kk, hist, &st->sel, tid, NS, sel_sync);
+          if (tid == 0) st->cnt = 0;
+          sel_sync();
+          for (int b0 = 0; b0 < n; b0 += NS) {
+            const int i = b0 + tid;
+            const uint64_t cv = i < n ? comp[i] : 0ull;
+            const bool take = i < n && cv >= thr;
+            const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
+            if (m == 0u) continue;
+            const int leader = __ffs(m) - 1;
+            int pos = 0;
+            if (lane == leader) pos = atomicAdd(&st->cnt, __popc(m));
+            pos = __shfl_sync(0xFFFFFFFFu, pos, leader) + __popc(m & ((1u << lane) - 1u));
+            if (take) {
+              kb[pos] = static_cast<uint32_t>(cv >> kIdxBits);
+              ib[pos] = composite_index(cv);
+            }
+          }
+          sel_sync();
+          if (tid == 0) {
+            st->tau_f = key_to_float(static_cast<uint32_t>(thr >> kIdxBits));
+            st->tau_set = 1;
+            st->strict = 1;
+            st->hist_on = 0;
+          }
+          sel_sync();
+        }
+        if (seg_end) {
+          if (tid == 0) {
+            p.cand_count[seg] = min(st->cnt, p.seg_cap);
+            p.cand_tau[seg] = st->tau_set ? ordered_key(st->tau_f) : 0u;
+          }
+          sel_sync();
+        }
       }
-      sync();
+      ++chunk_i;
+      if (++c == p.chunks_per_row) {
+        c = 0;
+        ++u;
+      }
+      if (++stg == core.nstage) {
+        stg = 0;
+        phase ^= 1u;
+      }
     }
   });
 }
@@ -904,7 +1030,7 @@ Layout fused_layout(int RG, int n_max, int k, int B) {
   return L;
 }
 
-constexpr size_t kPFusedExtra = 2048 * sizeof(unsigned) + sizeof(SegStateP);
+constexpr size_t kPFusedExtra = 2048 * sizeof(unsigned) + sizeof(SelStateP);
 
 struct FusedLaunch {
   const ScanParams& p;
@@ -991,7 +1117,7 @@ kvs_status fathom_scan_topk_launch(ScanParams p, void* ws, const int32_t* slot_m
     const size_t smem = prmt_smem_bytes(p.B, p.nstage, kPFusedExtra);
     cudaFuncSetAttribute(fathom_scan_topk_prmt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(smem));
-    fathom_scan_topk_prmt_kernel<<<L.grid, kPThreads, smem, s>>>(p);
+    fathom_scan_topk_prmt_kernel<<<L.grid, kPThreadsStaged, smem, s>>>(p);
     st = check_launch("decode_step(scan+topk, prmt)");
   } else {
     p.cand_tau = nullptr;

@@ -241,7 +241,7 @@ def test_decode_step_tiny_config(kvs):
     assert int(step.misses[0, 0]) == round(0.2 * 256)
 
 
-@pytest.mark.parametrize("B", [68, 92, 136, 512])
+@pytest.mark.parametrize("B", [1, 20, 68, 92, 136, 512])
 def test_decode_step_ragged_batch(kvs, B):
     nl = [20000, 7777, 2048, 1000]
     ref, step = _decode_case(kvs, 4, 2, 4, nl, 20000, B, 2048, 4096, seed=B)
