@@ -26,11 +26,13 @@ struct ScanParams {
   int warps;        // consumer warps per block (8 or 12); a chunk is 16 * warps words
   int chunks_per_row;
   float* scores;  // unfused output [RG][n_max]
+  float* gmax;    // optional: max score of each 16-key group [RG][ceil(n_max / 16)] (-inf if none valid)
   int32_t* dev_status;
   int nstage;  // pipeline depth (set by the launcher from the shared memory budget)
   // fused top-k candidates (scan_topk.cu)
   int k;
-  int segs_per_row, seg_cap;
+  int segs_per_row, seg_cap;  // candidate lists per row, and entries per list
+  int lists_per_seg;          // lists of one (block, row) segment: 1, or one per scoring warp
   int cand_cap, trim_at;  // per-block candidate capacity, and the count that triggers a trim
   uint32_t* cbuf_key;   // [grid][2][cap] per-block candidate buffers: score keys
   int32_t* cbuf_idx;    //                                             indices

@@ -95,12 +95,18 @@ struct LutLaunch {
 // Plans of at most 144 planes: the byte-indexed lookup core (scan_prmt.cuh).
 // Thread t writes the 16 consecutive scores of its half plane word.
 __global__ void __launch_bounds__(kPThreads, 1) fathom_scan_prmt_kernel(ScanParams p) {
-  ScanCoreP<false> core(p);
-  core.run([&](int u, int c, int nr, const float (&acc)[kPKeys], int t, unsigned char*) {
-    const int i0 = ScanCoreP<false>::key0(c, t);
+  ScanCoreP core(p);
+  core.run([&](int u, int c, int nr, const float (&acc)[kPKeys], int t) {
+    const int i0 = ScanCoreP::key0(c, t);
     if (i0 >= p.n_max) return;
     float* out = p.scores + static_cast<size_t>(u) * p.n_max;
     const float ninf = -__int_as_float(0x7f800000);
+    if (p.gmax) {
+      float m = ninf;
+#pragma unroll
+      for (int j = 0; j < kPKeys; ++j) m = fmaxf(m, i0 + j < nr ? acc[j] : ninf);
+      p.gmax[static_cast<size_t>(u) * ((p.n_max + kPKeys - 1) / kPKeys) + i0 / kPKeys] = m;
+    }
     if (i0 + kPKeys <= p.n_max && (p.n_max & 3) == 0) {
 #pragma unroll
       for (int j = 0; j < kPKeys; j += 4) {

@@ -49,9 +49,7 @@ namespace kvs {
 
 constexpr int kPWarps = 8;                      // consumer warps
 constexpr int kPProd = 4;                       // producer warps
-constexpr int kPSel = 4;                        // selector warps of the staged (fused top-k) mode
 constexpr int kPThreads = 32 * (kPWarps + kPProd);
-constexpr int kPThreadsStaged = 32 * (kPWarps + kPProd + kPSel);
 constexpr int kPKeys = 16;                      // keys per consumer thread (half a word)
 constexpr int kPChunkWords = 16 * kPWarps;      // plane words per chunk (4,096 keys)
 constexpr int kPRowBytes = 4 * kPChunkWords;    // one staged plane segment
@@ -132,12 +130,6 @@ __device__ __forceinline__ void partial_transpose16(uint32_t (&x)[16]) {
   }
 }
 
-// STAGED = false: the consumers run the epilogue themselves and release each
-// slot. STAGED = true: the consumers only write their 16 scores per thread
-// into their own column band of the slot (rows 0..31: lane L's 16 scores at
-// row L, bytes 64 * warp ..) and signal `scored`; kPSel selector warps consume
-// the scores and release the slot to the producers.
-template <bool STAGED>
 struct ScanCoreP {
   static constexpr int KEYS = kPKeys;
   static constexpr int CHUNK_WORDS = kPChunkWords;
@@ -153,7 +145,6 @@ struct ScanCoreP {
   uint32_t stage0;  // shared offset of slot 0 (relative to g_scan_smem)
   uint64_t* full;
   uint64_t* empty;
-  uint64_t* scored;
   int* abort_flag;
 
   __device__ explicit ScanCoreP(const ScanParams& params) : p(params) {
@@ -163,8 +154,7 @@ struct ScanCoreP {
     stage0 = kPTableBytes + kPZeroBytes;
     full = reinterpret_cast<uint64_t*>(g_scan_smem + stage0 + nstage * slot_bytes);
     empty = full + nstage;
-    scored = empty + nstage;
-    abort_flag = reinterpret_cast<int*>(scored + nstage);
+    abort_flag = reinterpret_cast<int*>(empty + nstage);
   }
 
   __device__ unsigned char* extra() const {
@@ -177,19 +167,6 @@ struct ScanCoreP {
   }
 
   __device__ static void sync() { consumer_sync<kPWarps>(); }
-
-  // Barrier of the consumer threads that also returns the OR of their
-  // predicates (the same value in every thread).
-  __device__ static bool sync_or(bool pred) {
-    int r;
-    asm volatile(
-        "{\n .reg .pred p, q;\n setp.ne.s32 p, %1, 0;\n bar.red.or.pred q, 1, %2, p;\n"
-        " selp.s32 %0, 1, 0, q;\n}\n"
-        : "=r"(r)
-        : "r"(pred ? 1 : 0), "n"(32 * kPWarps)
-        : "memory");
-    return r != 0;
-  }
 
   // Producer warp j (0..3) stages planes j, j + 4, j + 8, ... of every chunk.
   __device__ void produce(int beg, int end) {
@@ -377,10 +354,10 @@ struct ScanCoreP {
     }
   }
 
-  // epi(u, c, nr, acc, t, slot) runs in the consumers after each chunk (not
-  // STAGED); sel(beg, end) runs in the selector warps (STAGED).
-  template <typename Epi, typename Sel>
-  __device__ void run(Epi&& epi, Sel&& sel) {
+  // epi(u, c, nr, acc, t) runs in every consumer thread after each chunk c of
+  // row u (acc: its 16 scores; nr: the row's length).
+  template <typename Epi>
+  __device__ void run(Epi&& epi) {
     const int chunks = p.RG * p.chunks_per_row;
     const int beg = static_cast<int>(static_cast<long long>(blockIdx.x) * chunks / gridDim.x);
     const int end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * chunks / gridDim.x);
@@ -388,17 +365,12 @@ struct ScanCoreP {
     if (threadIdx.x == 0) {
       for (int i = 0; i < nstage; ++i) {
         mbar_init(&full[i], 32 * kPProd);
-        mbar_init(&empty[i], STAGED ? kPSel : kPWarps);
-        mbar_init(&scored[i], kPWarps);
+        mbar_init(&empty[i], kPWarps);
       }
       *abort_flag = 0;
       asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     __syncthreads();
-    if (warp >= kPWarps + kPProd) {
-      if constexpr (STAGED) sel(beg, end);
-      return;
-    }
     if (warp >= kPWarps) {
       produce(beg, end);
       return;
@@ -435,24 +407,8 @@ struct ScanCoreP {
         if (GB > 0) set_pass(soff, GB, lb, acc);
       }
       __syncwarp();
-      if constexpr (STAGED) {
-        // this warp's band of the slot (only this warp read it): lane L's
-        // scores in row L
-        if (!dead) {
-          float4* row = reinterpret_cast<float4*>(g_scan_smem + soff + lane * kPRowBytes + 64 * warp);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            row[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&scored[st]);
-        }
-      } else {
-        epi(u, c, nr, acc, static_cast<int>(threadIdx.x), g_scan_smem + soff);
-        if (!dead) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[st]);
-        }
-      }
+      if (!dead && lane == 0) mbar_arrive(&empty[st]);
+      epi(u, c, nr, acc, static_cast<int>(threadIdx.x));
       if (++c == p.chunks_per_row) {
         c = 0;
         ++u;
@@ -462,11 +418,6 @@ struct ScanCoreP {
         phase ^= 1u;
       }
     }
-  }
-
-  template <typename Epi>
-  __device__ void run(Epi&& epi) {
-    run(epi, [](int, int) {});
   }
 };
 

@@ -33,7 +33,6 @@ namespace {
 constexpr int kIdxBits = 21;
 constexpr uint32_t kIdxMask = (1u << kIdxBits) - 1u;
 constexpr int kCandCap = 16384;  // per-block candidate buffer entries in global memory
-constexpr int kPCandCap = 24576; // per-segment candidates of the byte-indexed fused scan
 
 __device__ __forceinline__ uint64_t make_composite(uint32_t key, int idx) {
   return (static_cast<uint64_t>(key) << kIdxBits) |
@@ -420,394 +419,6 @@ __global__ void KVS_SCAN_BOUNDS(G, b, W) fathom_scan_topk_kernel(ScanParams p) {
   });
 }
 
-// ---------------------------------------------------------------------------
-// Fused scan + top-k on the byte-indexed lookup core (plans of <= 144 planes).
-//
-// The eight scoring warps only write each chunk's 4,096 scores into the
-// consumed stage slot (scan_prmt.cuh, staged mode); four selector warps, one
-// per scheduler, read them there (two scoring warps' bands each) and keep the
-// segment's candidates, so the latency of the selection never stalls the
-// scoring warps. A segment's candidates are appended straight into its output
-// region (capacity kPCandCap) as (order-preserving score key, index): a lane
-// marks which of its 32 scores are at or above the running threshold tau, the
-// warp takes its positions with one shuffle scan and one shared atomic, and
-// only the marked scores are read again and written.
-//
-// tau: the segment's first chunk (when it holds >= k valid keys) is binned
-// linearly over [min, max] of its scores into 2048 bins; tau becomes the
-// smallest score in the bin holding the k-th largest, so exactly the keys of
-// that bin and above are held. Every later appended key is counted in its
-// bin. Whenever the held count has grown by k/4 since the last raise, the one
-// selector warp that moves the raise mark (a compare-and-swap) finds the bin b
-// holding the k-th largest held key and raises tau to the lower edge of bin
-// b - 1 (one bin of margin against rounding). The counts it reads may lag
-// appends still in flight, so they are lower bounds: at least k held keys are
-// >= tau at all times and the held set is a superset of the segment's top-k.
-// A segment of n keys appends about k (1 + ln(n / 4096)) keys (~9,000 for
-// 113K keys, ~10,500 for 230K). Every second chunk the selectors check the
-// fill; near capacity (ties, degenerate ranges) the held set is cut to exactly
-// the k best by (score, index) and, since later keys have larger indices, only
-// keys strictly above the k-th score are appended afterwards. The segment's
-// final tau is stored beside its count; the merge drops entries below it.
-struct SelStateP {
-  int cnt, tau_set, strict, hist_on, next_raise;
-  float tau_f, lo, w, inv_w;
-  float red_min[kPSel], red_max[kPSel];
-  SelectState sel;
-};
-
-__device__ __forceinline__ int score_bin(float s, float lo, float inv_w) {
-  return min(2047, max(0, static_cast<int>((s - lo) * inv_w)));
-}
-
-// One warp: the bin holding the k-th largest count of hist (from the top), or
-// -1 when the histogram holds fewer than k. Lane l first sums bins
-// [2048 - 64 (l + 1), 2048 - 64 l) (16-byte reads in a lane-rotated order),
-// then the lane holding the rank is resolved two bins per lane.
-__device__ __forceinline__ int warp_kth_bin(const unsigned* hist, int k, int lane) {
-  const uint4* h4 = reinterpret_cast<const uint4*>(hist);
-  const int q0 = 512 - 16 * (lane + 1);
-  unsigned sum = 0;
-#pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const uint4 v = h4[q0 + ((e + lane) & 15)];
-    sum += v.x + v.y + v.z + v.w;
-  }
-  unsigned incl = sum;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const unsigned o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-    if (lane >= d) incl += o;
-  }
-  const unsigned hit = __ballot_sync(0xFFFFFFFFu, incl >= static_cast<unsigned>(k));
-  if (hit == 0u) return -1;
-  const int L = __ffs(hit) - 1;
-  const unsigned krem = static_cast<unsigned>(k) - __shfl_sync(0xFFFFFFFFu, incl - sum, L);
-  const int b_hi = 2048 - 64 * L - 1 - 2 * lane;
-  const unsigned c_hi = hist[b_hi], c_lo = hist[b_hi - 1];
-  const unsigned c2 = c_hi + c_lo;
-  unsigned incl2 = c2;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const unsigned o = __shfl_up_sync(0xFFFFFFFFu, incl2, d);
-    if (lane >= d) incl2 += o;
-  }
-  const unsigned hit2 = __ballot_sync(0xFFFFFFFFu, incl2 >= krem);
-  const int l2 = hit2 ? __ffs(hit2) - 1 : 31;
-  const unsigned before = __shfl_sync(0xFFFFFFFFu, incl2 - c2, l2);
-  const unsigned top_cnt = __shfl_sync(0xFFFFFFFFu, c_hi, l2);
-  const int bb = 2048 - 64 * L - 1 - 2 * l2;
-  return before + top_cnt >= krem ? bb : bb - 1;
-}
-
-// Barrier of the selector warps only; and the same returning the OR of a predicate.
-__device__ __forceinline__ void sel_sync() {
-  asm volatile("bar.sync 2, %0;\n" ::"n"(32 * kPSel) : "memory");
-}
-__device__ __forceinline__ bool sel_sync_or(bool pred) {
-  int r;
-  asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.s32 p, %1, 0;\n bar.red.or.pred q, 2, %2, p;\n"
-      " selp.s32 %0, 1, 0, q;\n}\n"
-      : "=r"(r)
-      : "r"(pred ? 1 : 0), "n"(32 * kPSel)
-      : "memory");
-  return r != 0;
-}
-
-__global__ void __launch_bounds__(kPThreadsStaged, 1) fathom_scan_topk_prmt_kernel(ScanParams p) {
-  using Core = ScanCoreP<true>;
-  Core core(p);
-  unsigned* hist = reinterpret_cast<unsigned*>(core.extra());
-  SelStateP* st = reinterpret_cast<SelStateP*>(hist + 2048);
-  volatile SelStateP* vst = st;
-  core.run([](int, int, int, const float (&)[kPKeys], int, unsigned char*) {}, [&](int beg, int end) {
-    constexpr int NS = 32 * kPSel;
-    constexpr int CK = 32 * kPChunkWords;  // keys per chunk
-    const int lane = threadIdx.x & 31;
-    const int sw = (threadIdx.x >> 5) - (kPWarps + kPProd);
-    const int tid = 32 * sw + lane;
-    const long long C = static_cast<long long>(p.RG) * p.chunks_per_row;
-    const int last_chunk = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * C / gridDim.x) - 1;
-    const int raise_step = max(256, p.k / 4);
-    const float pinf = __int_as_float(0x7f800000), ninf = -pinf;
-    // lane's place in a chunk: iteration e reads row 4e + (lane >> 3), 16 bytes
-    // q4 = lane & 7 of this warp's 128-byte part (scoring warps 2 sw, 2 sw + 1)
-    const int q4 = lane & 7;
-    const int cw = 2 * sw + (q4 >> 2);  // scoring warp whose scores these are
-    int u = beg / p.chunks_per_row, c = beg % p.chunks_per_row, stg = 0;
-    uint32_t phase = 0u;
-    int chunk_i = 0, seg_u = -1;
-    size_t seg = 0;
-    bool fresh = false, dead = false;
-    for (int it = beg; it < end; ++it) {
-      const int nr = p.n[u / p.Gheads];
-      if (u != seg_u) {
-        seg = static_cast<size_t>(u) * p.segs_per_row +
-              (static_cast<int>(blockIdx.x) -
-               block_of_chunk(static_cast<long long>(u) * p.chunks_per_row, C, gridDim.x));
-        seg_u = u;
-        fresh = true;
-        if (tid == 0) {
-          st->cnt = 0;
-          st->tau_set = 0;
-          st->strict = 0;
-          st->hist_on = 0;
-        }
-        sel_sync();
-      }
-      if (!dead && !mbar_wait(&core.scored[stg], phase)) {
-        core.fail_timeout();
-        dead = true;
-      }
-      unsigned char* slot = g_scan_smem + core.stage0 + stg * core.slot_bytes;
-      uint32_t* kb = p.cand_key + seg * p.seg_cap;
-      int32_t* ib = p.cand_idx + seg * p.seg_cap;
-      // this lane's 32 scores and their validity; score j is key
-      // kbase0 + 64 (j >> 2) + (j & 3)
-      const int kbase0 = 32 * (c * kPChunkWords + 16 * cw + (lane >> 4)) + 16 * ((lane >> 3) & 1) + 4 * (q4 & 3);
-      float4 v[8];
-      uint32_t valid = 0u;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int r = 4 * e + (lane >> 3);
-        v[e] = *reinterpret_cast<const float4*>(slot + r * kPRowBytes + 128 * sw + 16 * q4);
-        const int nv = nr - (kbase0 + 64 * e);
-        valid |= (nv >= 4 ? 15u : (nv <= 0 ? 0u : ((1u << nv) - 1u))) << (4 * e);
-      }
-      auto score = [&](int j) -> float {
-        const float4 f = v[j >> 2];
-        const int cc = j & 3;
-        return cc == 0 ? f.x : (cc == 1 ? f.y : (cc == 2 ? f.z : f.w));
-      };
-      // 0. the segment's first chunk: tau from its own scores (its held keys are
-      // then already counted in the histogram)
-      bool binned_now = false;
-      if (fresh) {
-        fresh = false;
-        if (nr - 32 * c * kPChunkWords >= p.k) {
-          float mn = pinf, mx = ninf;
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if ((valid >> j) & 1u) {
-              mn = fminf(mn, score(j));
-              mx = fmaxf(mx, score(j));
-            }
-          for (int d = 16; d > 0; d >>= 1) {
-            mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, d));
-            mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, d));
-          }
-          if (lane == 0) {
-            st->red_min[sw] = mn;
-            st->red_max[sw] = mx;
-          }
-          for (int b = tid; b < 2048; b += NS) hist[b] = 0;
-          sel_sync();
-          float lo = st->red_min[0], hi = st->red_max[0];
-#pragma unroll
-          for (int q = 1; q < kPSel; ++q) {
-            lo = fminf(lo, st->red_min[q]);
-            hi = fmaxf(hi, st->red_max[q]);
-          }
-          const float w = (hi - lo) * (1.0f / 2048.0f);
-          const float mag = fmaxf(fabsf(lo), fabsf(hi));
-          // bins are usable when one bin is well above the rounding of scores
-          if (hi > lo && w > 16.0f * mag * 5.96e-8f) {  // the same in every selector thread
-            const float inv_w = 2048.0f / (hi - lo);
-            binned_now = true;
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if ((valid >> j) & 1u) atomicAdd(&hist[score_bin(score(j), lo, inv_w)], 1u);
-            sel_sync();
-            const int bstar = warp_kth_bin(hist, p.k, lane);  // the same in every warp
-            // tau = the smallest score in bin bstar (exact: bins are monotone in the score)
-            float bmin = pinf;
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (((valid >> j) & 1u) && score_bin(score(j), lo, inv_w) == bstar) bmin = fminf(bmin, score(j));
-            for (int d = 16; d > 0; d >>= 1) bmin = fminf(bmin, __shfl_xor_sync(0xFFFFFFFFu, bmin, d));
-            sel_sync();  // every warp has read the histogram
-            // the held keys are exactly bins >= bstar: clear the rest of the histogram
-            for (int b = tid; b < bstar; b += NS) hist[b] = 0;
-            if (lane == 0) st->red_min[sw] = bmin;
-            sel_sync();
-            if (tid == 0) {
-              float tm = st->red_min[0];
-              for (int q = 1; q < kPSel; ++q) tm = fminf(tm, st->red_min[q]);
-              st->tau_f = tm;
-              st->tau_set = 1;
-              st->hist_on = 1;
-              st->lo = lo;
-              st->w = w;
-              st->inv_w = inv_w;
-              st->next_raise = p.k + raise_step;
-            }
-            sel_sync();
-          }
-        }
-      }
-
-      // 1. keys at or above tau join the segment's candidates
-      const bool count_bins = vst->hist_on != 0 && !binned_now;
-      float tau = ninf;
-      if (vst->tau_set) {
-        tau = vst->tau_f;
-        if (vst->strict) tau = nextafterf(tau, pinf);  // strictly above the cut's k-th score
-      }
-      uint32_t mask = 0u;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) mask |= score(j) >= tau ? (1u << j) : 0u;
-      mask &= valid;
-      // appends, in two halves of 16 keys per lane: lane L first writes its
-      // passing (score, key) pairs densely into row L of this warp's part of
-      // the slot (128 bytes: 16 pairs; its scores are in registers now), then
-      // the warp writes them out one pair per lane (each lane finds the pair's
-      // source lane by binary search over the lanes' offsets), with one shared
-      // atomic per half for their positions
-      __syncwarp();
-      int new_cnt = -1;
-      unsigned char* mine = slot + lane * kPRowBytes + 128 * sw;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const uint32_t hm = (mask >> (16 * half)) & 0xFFFFu;
-        const int cnt = __popc(hm);
-        int incl = cnt;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-          const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-          if (lane >= d) incl += o;
-        }
-        const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-        if (total == 0) continue;
-        uint32_t woff = 0u;
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int j = 16 * half + jj;
-          if ((hm >> jj) & 1u) {
-            *reinterpret_cast<uint2*>(mine + woff) = make_uint2(
-                __float_as_uint(score(j)), static_cast<uint32_t>(kbase0 + 64 * (j >> 2) + (j & 3)));
-            woff += 8u;
-          }
-        }
-        int base = 0;
-        if (lane == 0) base = atomicAdd(&st->cnt, total);
-        base = __shfl_sync(0xFFFFFFFFu, base, 0);
-        new_cnt = base + total;
-        const int excl = incl - cnt;
-        __syncwarp();
-        const float lo = st->lo, inv_w = st->inv_w;
-        for (int f0 = 0; f0 < total; f0 += 32) {
-          const int f = f0 + lane;
-          // source lane: the last lane whose exclusive offset is <= f
-          int src = 0;
-#pragma unroll
-          for (int step = 16; step > 0; step >>= 1) {
-            const int probe = src + step;
-            if (__shfl_sync(0xFFFFFFFFu, excl, probe) <= f) src = probe;
-          }
-          const int rank = f - __shfl_sync(0xFFFFFFFFu, excl, src);
-          if (f < total) {
-            const uint2 e = *reinterpret_cast<const uint2*>(slot + src * kPRowBytes + 128 * sw + 8 * rank);
-            const float sc = __uint_as_float(e.x);
-            if (base + f < p.seg_cap) {
-              kb[base + f] = ordered_key(sc);
-              ib[base + f] = static_cast<int32_t>(e.y);
-            }
-            if (count_bins) atomicAdd(&hist[score_bin(sc, lo, inv_w)], 1u);
-          }
-        }
-        __syncwarp();
-      }
-      // the warp that moves the raise mark raises tau from the histogram
-      if (count_bins && new_cnt >= 0) {
-        int won = 0;
-        if (lane == 0) {
-          const int mark = vst->next_raise;
-          won = new_cnt >= mark && atomicCAS(&st->next_raise, mark, new_cnt + raise_step) == mark;
-        }
-        if (__shfl_sync(0xFFFFFFFFu, won, 0)) {
-          const int b = warp_kth_bin(hist, p.k, lane);
-          if (lane == 0 && b >= 1) {
-            const float edge = st->lo + static_cast<float>(b - 1) * st->w;
-            if (edge > vst->tau_f) vst->tau_f = edge;
-          }
-        }
-      }
-
-      // the slot goes back to the producers; rows that are padding planes
-      // (B < 32) must be zero again
-      if (p.B < 32) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if (4 * e + (lane >> 3) >= p.B)
-            *reinterpret_cast<float4*>(slot + (4 * e + (lane >> 3)) * kPRowBytes + 128 * sw + 16 * q4) =
-                make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-      __syncwarp();
-      if (!dead && lane == 0) mbar_arrive(&core.empty[stg]);
-
-      // 3. at the segment's end (publish), and every second chunk (the buffer
-      // may take two more chunks of appends before it must be cut)
-      const bool seg_end = c == p.chunks_per_row - 1 || u * p.chunks_per_row + c == last_chunk;
-      if (seg_end || (chunk_i & 1)) {
-        sel_sync();  // every warp's appends of this chunk are done
-        // one decision for all: the count is read after the barrier, and no warp
-        // appends again before every thread has read it
-        if (sel_sync_or(!seg_end && st->cnt > p.seg_cap - 2 * CK)) {
-          // exact cut to the k best by (score key, index)
-          const int n = st->cnt;
-          uint64_t* comp = p.cbuf_comp + static_cast<size_t>(blockIdx.x) * p.seg_cap;
-          for (int i = tid; i < n; i += NS) comp[i] = make_composite(kb[i], ib[i]);
-          sel_sync();
-          const int kk = min(p.k, n);
-          const uint64_t thr = select_kth_composite(comp, n, kk, hist, &st->sel, tid, NS, sel_sync);
-          if (tid == 0) st->cnt = 0;
-          sel_sync();
-          for (int b0 = 0; b0 < n; b0 += NS) {
-            const int i = b0 + tid;
-            const uint64_t cv = i < n ? comp[i] : 0ull;
-            const bool take = i < n && cv >= thr;
-            const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
-            if (m == 0u) continue;
-            const int leader = __ffs(m) - 1;
-            int pos = 0;
-            if (lane == leader) pos = atomicAdd(&st->cnt, __popc(m));
-            pos = __shfl_sync(0xFFFFFFFFu, pos, leader) + __popc(m & ((1u << lane) - 1u));
-            if (take) {
-              kb[pos] = static_cast<uint32_t>(cv >> kIdxBits);
-              ib[pos] = composite_index(cv);
-            }
-          }
-          sel_sync();
-          if (tid == 0) {
-            st->tau_f = key_to_float(static_cast<uint32_t>(thr >> kIdxBits));
-            st->tau_set = 1;
-            st->strict = 1;
-            st->hist_on = 0;
-          }
-          sel_sync();
-        }
-        if (seg_end) {
-          if (tid == 0) {
-            p.cand_count[seg] = min(st->cnt, p.seg_cap);
-            p.cand_tau[seg] = st->tau_set ? ordered_key(st->tau_f) : 0u;
-          }
-          sel_sync();
-        }
-      }
-      ++chunk_i;
-      if (++c == p.chunks_per_row) {
-        c = 0;
-        ++u;
-      }
-      if (++stg == core.nstage) {
-        stg = 0;
-        phase ^= 1u;
-      }
-    }
-  });
-}
-
 // One block per (r, g): gather the segments' candidates, select the k best,
 // emit their indices in ascending order, look up their slots. 1024 threads.
 // The ascending order comes from a bitmap over the row's key indices (in the
@@ -829,8 +440,8 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(
     int32_t* __restrict__ misses) {
   __shared__ unsigned hist[2048];
   __shared__ SelectState sel;
-  __shared__ int seg_count[64], seg_off[65];
-  __shared__ uint32_t seg_tau[64];
+  __shared__ int seg_count[512], seg_off[513];
+  __shared__ uint32_t seg_tau[512];
   __shared__ int kept_total;
   __shared__ int wsum[kMergeThreads / 32];
   __shared__ int miss_warp[kMergeThreads / 32];
@@ -843,7 +454,7 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(
   const long long C = static_cast<long long>(p.RG) * p.chunks_per_row;
   const int b0 = block_of_chunk(static_cast<long long>(u) * p.chunks_per_row, C, scan_grid);
   const int b1 = block_of_chunk(static_cast<long long>(u + 1) * p.chunks_per_row - 1, C, scan_grid);
-  const int segs = b1 - b0 + 1;
+  const int segs = (b1 - b0 + 1) * p.lists_per_seg;
   if (t < segs) {
     seg_count[t] = p.cand_count[static_cast<size_t>(u) * p.segs_per_row + t];
     seg_tau[t] = p.cand_tau ? p.cand_tau[static_cast<size_t>(u) * p.segs_per_row + t] : 0u;
@@ -992,6 +603,330 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------
+// Top-k of one (request, KV head) row from its scores and 16-key group maxima
+// (the byte-indexed scan writes both). One block of 1,024 threads per row.
+//  A. T = (a lower bound of) the kk-th largest group maximum: each group
+//     maximum is a distinct key, so at least kk keys are >= T and the row's
+//     kk-th largest score is >= T. Groups whose maximum is below T hold no
+//     selected key and are never read again (about a quarter of the groups
+//     remain for Gaussian-like scores).
+//  B. Radix select (11/11/10 bits of the order-preserving key) over the keys
+//     >= T of the remaining groups: either a whole key cell holds the last
+//     selected ranks (select every key >= its lower edge: exactly kk keys), or
+//     the exact kk-th largest key K* (select the keys > K*, and of the keys
+//     equal to K* the lowest indices).
+//  C. The selected keys are marked in a bitmap over the row, ties by index
+//     order (groups are visited in index order in rounds of 1,024 with one
+//     block-wide scan per round), and emitted in ascending order with the
+//     slot of each and the row's miss count.
+constexpr int kTkThreads = 1024;
+
+struct TkState {
+  int wsum[32], res[2];
+  uint32_t prefix, mask;
+  int krem, done, gt;
+  int tie_base;
+  int miss_warp[32];
+};
+
+// Block-wide radix select of the kk-th largest key over the keys enumerated by
+// each(visit) (every thread visits its own share; the same set each pass).
+// Returns the cell or key; *whole is true when every key >= the returned value
+// is selected (exactly kk of them), false when it is the exact kk-th key and
+// *gt keys lie strictly above it.
+template <typename Each>
+__device__ uint32_t radix_kth_key(Each&& each, int kk, unsigned* hist, TkState* st, bool* whole, int* gt) {
+  const int t = threadIdx.x;
+  if (t == 0) {
+    st->prefix = 0u;
+    st->mask = 0u;
+    st->krem = kk;
+    st->done = 0;
+    st->gt = 0;
+  }
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const uint32_t dmask = pass < 2 ? 2047u : 1023u;
+    for (int b = t; b < 2048; b += kTkThreads) hist[b] = 0;
+    __syncthreads();
+    const uint32_t prefix = st->prefix, mask = st->mask;
+    each([&](uint32_t key) {
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+    });
+    __syncthreads();
+    find_bin_from_top(hist, static_cast<int>(dmask) + 1, st->krem, st->wsum, st->res, t, kTkThreads,
+                      [] { __syncthreads(); });
+    if (t == 0) {
+      const int bin = st->res[0];
+      st->prefix = prefix | (static_cast<uint32_t>(bin) << shift);
+      st->mask = mask | (dmask << shift);
+      st->krem -= st->res[1];
+      st->gt += st->res[1];
+      st->done = st->krem == static_cast<int>(hist[bin]) ? 1 : (pass == 2 ? 2 : 0);
+    }
+    __syncthreads();
+    if (st->done) break;
+  }
+  *whole = st->done == 1;
+  *gt = st->gt;
+  return st->prefix;
+}
+
+constexpr int kTkMaxGroups = 65536;  // group maxima kept in shared memory (16-bit prefixes)
+constexpr int kTkCandGroups = 6144;  // candidate groups, and candidate keys, on chip
+constexpr int kTkCandKeys = 6144;
+constexpr size_t kTkSmem = kTkMaxGroups * sizeof(uint16_t) + kTkCandGroups * sizeof(int) +
+                           kTkCandKeys * sizeof(uint2);
+
+// Block-wide exclusive prefix of c over the threads (in thread order); returns
+// it and the block total.
+__device__ __forceinline__ int block_excl_scan(int c, TkState* st, int* total) {
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  int incl = c;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+    if (lane >= d) incl += o;
+  }
+  if (lane == 31) st->wsum[warp] = incl;
+  __syncthreads();
+  const int before = __reduce_add_sync(0xFFFFFFFFu, lane < warp ? st->wsum[lane] : 0);
+  *total = __reduce_add_sync(0xFFFFFFFFu, st->wsum[lane]);
+  __syncthreads();
+  return before + incl - c;
+}
+
+__global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(
+    const float* __restrict__ scores, const float* __restrict__ gmax, const int32_t* __restrict__ n,
+    int Gheads, int n_max, int k, uint32_t* __restrict__ bitmap, const int32_t* __restrict__ slot_map,
+    int32_t* __restrict__ idx, int32_t* __restrict__ slots, int32_t* __restrict__ misses) {
+  __shared__ unsigned hist[2048];
+  __shared__ TkState st;
+  extern __shared__ __align__(16) unsigned char tk_smem[];
+  uint16_t* gk = reinterpret_cast<uint16_t*>(tk_smem);                      // [kTkMaxGroups]
+  int* cg = reinterpret_cast<int*>(tk_smem + kTkMaxGroups * sizeof(uint16_t));  // [kTkCandGroups]
+  uint2* ck = reinterpret_cast<uint2*>(cg + kTkCandGroups);                 // [kTkCandKeys] (key, index)
+  constexpr int NG = 16;  // keys per group
+  const float ninf = -__int_as_float(0x7f800000);
+  const int u = blockIdx.x;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int nr = min(n[u / Gheads], n_max);
+  const int kk = min(k, nr);
+  const int ldg = (n_max + NG - 1) / NG;
+  const int m = (nr + NG - 1) / NG;
+  const float* sc = scores + static_cast<size_t>(u) * n_max;
+  const float* gm = gmax + static_cast<size_t>(u) * ldg;
+  const bool vec = (n_max & 3) == 0;
+  const int words = bitmap_words(n_max);
+  uint32_t* bm = bitmap + static_cast<size_t>(u) * words;
+  for (int w = 4 * t; w < words; w += 4 * kTkThreads)
+    *reinterpret_cast<uint4*>(bm + w) = make_uint4(0u, 0u, 0u, 0u);
+
+  // the 16 scores of group g (invalid keys: -inf, written by the scan)
+  auto load_group = [&](int g, float (&v)[NG]) {
+    const float* src = sc + static_cast<size_t>(g) * NG;
+    if (vec && g * NG + NG <= n_max) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 f = __ldg(reinterpret_cast<const float4*>(src) + q);
+        v[4 * q] = f.x;
+        v[4 * q + 1] = f.y;
+        v[4 * q + 2] = f.z;
+        v[4 * q + 3] = f.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < NG; ++j) v[j] = g * NG + j < n_max ? __ldg(src + j) : ninf;
+    }
+  };
+
+  bool whole = true;
+  int gt = 0;
+  uint32_t key_cut = 0u;
+  int nck = -1;  // keys >= T on chip (-1: too many, the rows' scores are read again)
+  uint32_t T = 0u;
+  if (kk > 0 && m <= kTkMaxGroups) {
+    // A. the group maxima on chip as 16-bit key prefixes; T from them (at
+    // least kk maxima have a prefix >= T's, so at least kk keys are >= T)
+#pragma unroll 4
+    for (int g = t; g < m; g += kTkThreads) gk[g] = static_cast<uint16_t>(ordered_key(__ldg(gm + g)) >> 16);
+    __syncthreads();
+    if (kk <= m) {
+      bool wh;
+      int g0;
+      T = radix_kth_key([&](auto visit) {
+            for (int g = t; g < m; g += kTkThreads) visit(static_cast<uint32_t>(gk[g]) << 16);
+          }, kk, hist, &st, &wh, &g0) & 0xFFFF0000u;
+    }
+    // candidate groups in index order
+    int ncg = 0;
+    for (int r0 = 0; r0 < m; r0 += kTkThreads) {
+      const int g = r0 + t;
+      const int c = g < m && (static_cast<uint32_t>(gk[g]) << 16) >= T ? 1 : 0;
+      int tot;
+      const int pos = block_excl_scan(c, &st, &tot);
+      if (c && ncg + pos < kTkCandGroups) cg[ncg + pos] = g;
+      ncg += tot;
+    }
+    if (ncg <= kTkCandGroups) {
+      // keys >= T of the candidate groups, in index order (the groups' scores
+      // are loaded in one round per 1,024 groups)
+      nck = 0;
+      for (int r0 = 0; r0 < ncg; r0 += kTkThreads) {
+        const int e = r0 + t;
+        float v[NG];
+        uint32_t pass = 0u;
+        int g = 0;
+        if (e < ncg) {
+          g = cg[e];
+          load_group(g, v);
+#pragma unroll
+          for (int j = 0; j < NG; ++j)
+            if (g * NG + j < nr && ordered_key(v[j]) >= T) pass |= 1u << j;
+        }
+        int tot;
+        int pos = nck + block_excl_scan(__popc(pass), &st, &tot);
+        if (nck + tot <= kTkCandKeys) {
+          while (pass) {
+            const int j = __ffs(pass) - 1;
+            pass &= pass - 1u;
+            ck[pos++] = make_uint2(ordered_key(v[j]), static_cast<uint32_t>(g * NG + j));
+          }
+        }
+        nck += tot;
+      }
+      if (nck > kTkCandKeys) nck = -1;
+    }
+    __syncthreads();
+  }
+
+  if (kk > 0 && nck >= 0) {
+    // B. on chip: the kk-th largest candidate key
+    key_cut = radix_kth_key([&](auto visit) {
+                for (int e = t; e < nck; e += kTkThreads) visit(ck[e].x);
+              }, kk, hist, &st, &whole, &gt);
+    // C. mark the selected keys; ties by index (the list is in index order)
+    const int need = whole ? 0 : kk - gt;
+    int tie_base = 0;
+    for (int r0 = 0; r0 < nck; r0 += kTkThreads) {
+      const int e = r0 + t;
+      uint2 c = make_uint2(0u, 0u);
+      bool sel = false, tie = false;
+      if (e < nck) {
+        c = ck[e];
+        sel = whole ? c.x >= key_cut : c.x > key_cut;
+        tie = !whole && c.x == key_cut;
+      }
+      if (!whole) {
+        int tot;
+        const int rank = tie_base + block_excl_scan(tie ? 1 : 0, &st, &tot);
+        if (tie && rank < need) sel = true;
+        tie_base += tot;
+      }
+      if (sel) atomicOr(bm + (c.y >> 5), 1u << (c.y & 31));
+    }
+  } else if (kk > 0) {
+    // too many candidates for the chip: the same selection over the rows'
+    // scores in global memory (groups whose maximum is below T are skipped)
+    key_cut = radix_kth_key([&](auto visit) {
+                for (int g = t; g < m; g += kTkThreads) {
+                  if (ordered_key(__ldg(gm + g)) < T) continue;
+                  float v[NG];
+                  load_group(g, v);
+#pragma unroll
+                  for (int j = 0; j < NG; ++j)
+                    if (g * NG + j < nr) {
+                      const uint32_t key = ordered_key(v[j]);
+                      if (key >= T) visit(key);
+                    }
+                }
+              }, kk, hist, &st, &whole, &gt);
+    const int need = whole ? 0 : kk - gt;
+    int tie_base = 0;
+    for (int r0 = 0; r0 < m; r0 += kTkThreads) {
+      const int g = r0 + t;
+      uint32_t sel = 0u, tie = 0u;
+      if (g < m && ordered_key(__ldg(gm + g)) >= key_cut) {
+        float v[NG];
+        load_group(g, v);
+#pragma unroll
+        for (int j = 0; j < NG; ++j) {
+          if (g * NG + j >= nr) continue;
+          const uint32_t key = ordered_key(v[j]);
+          if (whole ? key >= key_cut : key > key_cut) sel |= 1u << j;
+          else if (!whole && key == key_cut) tie |= 1u << j;
+        }
+      }
+      if (!whole) {
+        int tot;
+        int rank = tie_base + block_excl_scan(__popc(tie), &st, &tot);
+        while (tie) {
+          const int j = __ffs(tie) - 1;
+          tie &= tie - 1u;
+          if (rank < need) sel |= 1u << j;
+          ++rank;
+        }
+        tie_base += tot;
+      }
+      if (sel) atomicOr(bm + (g >> 1), (g & 1) ? (sel << 16) : sel);
+    }
+  }
+  __syncthreads();
+  // ascending emission: thread t owns words [t * wpt, (t + 1) * wpt)
+  const int wpt = ((words + kTkThreads - 1) / kTkThreads + 3) & ~3;
+  const int w_beg = min(words, t * wpt), w_end = min(words, w_beg + wpt);
+  int cnt = 0;
+  for (int w = w_beg; w < w_end; w += 4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(bm + w);
+    cnt += __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
+  }
+  int incl = cnt;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+    if (lane >= d) incl += o;
+  }
+  if (lane == 31) st.wsum[warp] = incl;
+  __syncthreads();
+  const int before = __reduce_add_sync(0xFFFFFFFFu, lane < warp ? st.wsum[lane] : 0);
+  int pos = before + incl - cnt;
+  int32_t* irow = idx + static_cast<size_t>(u) * k;
+  for (int w = w_beg; w < w_end && cnt > 0; ++w) {
+    uint32_t bits = bm[w];
+    while (bits) {
+      const int bpos = __ffs(bits) - 1;
+      bits &= bits - 1u;
+      if (pos < k) irow[pos] = 32 * w + bpos;
+      ++pos;
+    }
+  }
+  __syncthreads();
+  const int chosen_total = min(__reduce_add_sync(0xFFFFFFFFu, st.wsum[lane]), kk);
+  int my_miss = 0;
+  for (int j = t; j < k; j += kTkThreads) {
+    int i = -1;
+    if (j < chosen_total)
+      i = irow[j];
+    else
+      irow[j] = -1;
+    int sl = -2;
+    if (i >= 0) {
+      sl = slot_map ? slot_map[static_cast<size_t>(u) * n_max + i] : -1;
+      my_miss += sl < 0 ? 1 : 0;
+    }
+    if (slots) slots[static_cast<size_t>(u) * k + j] = sl;
+  }
+  const int wm = __reduce_add_sync(0xFFFFFFFFu, my_miss);
+  if (lane == 0) st.miss_warp[warp] = wm;
+  __syncthreads();
+  if (t == 0 && misses) {
+    int mm = 0;
+    for (int e = 0; e < kTkThreads / 32; ++e) mm += st.miss_warp[e];
+    misses[u] = mm;
+  }
+}
+
 int fused_grid(int RG, int cpr) {
   const long long C = static_cast<long long>(RG) * cpr;
   return static_cast<int>(C < sm_count() ? C : sm_count());
@@ -1009,28 +944,23 @@ int fused_segs_per_row(int RG, int cpr, int grid) {
 }
 
 struct Layout {
-  int grid, cpr, segs, seg_cap;
+  int grid, cpr, segs, lists, list_cap;  // segments per row, candidate lists per segment
 };
 
-// Plans of <= 144 planes run the byte-indexed core, whose segments hold up to
-// kPCandCap candidates each; longer plans the group-table core (2k each).
+// Plans of more than 144 planes: the group-table core, one candidate list of
+// 2k per (block, row) segment.
 Layout fused_layout(int RG, int n_max, int k, int B) {
   Layout L{};
-  if (B <= kPMaxB) {
-    L.cpr = prmt_chunks_per_row(n_max);
-    L.seg_cap = kPCandCap;
-  } else {
-    int G, b, nsets;
-    scan_schedule(B, G, b, nsets);
-    L.cpr = scan_chunks_per_row(n_max, scan_warps(G, b));
-    L.seg_cap = 2 * k;
-  }
+  int G, b, nsets;
+  scan_schedule(B, G, b, nsets);
+  L.cpr = scan_chunks_per_row(n_max, scan_warps(G, b));
+  L.lists = 1;
+  L.list_cap = 2 * k;
   L.grid = fused_grid(RG, L.cpr);
   L.segs = L.grid > 0 ? fused_segs_per_row(RG, L.cpr, L.grid) : 1;
   return L;
 }
 
-constexpr size_t kPFusedExtra = 2048 * sizeof(unsigned) + sizeof(SelStateP);
 
 struct FusedLaunch {
   const ScanParams& p;
@@ -1075,17 +1005,25 @@ bool fused_topk_supported(int n_max, int k, int B) {
 }
 
 size_t fused_ws_bytes(int RG, int n_max, int k, int B) {
+  if (B <= kPMaxB) {
+    WsCarver c(nullptr);
+    c.take<float>(static_cast<size_t>(RG) * n_max);
+    c.take<float>(static_cast<size_t>(RG) * ((n_max + kPKeys - 1) / kPKeys));
+    c.take<uint32_t>(static_cast<size_t>(RG) * bitmap_words(n_max));
+    return c.used;
+  }
   const Layout L = fused_layout(RG, n_max, k, B);
+  const size_t lists = static_cast<size_t>(RG) * L.segs * L.lists;
+  const size_t comp = static_cast<size_t>(kCandCap > L.lists * L.list_cap ? kCandCap : L.lists * L.list_cap);
   WsCarver c(nullptr);
-  const size_t cap = static_cast<size_t>(kCandCap > L.seg_cap ? kCandCap : L.seg_cap);
   c.take<uint32_t>(static_cast<size_t>(L.grid) * kCandCap);
   c.take<int32_t>(static_cast<size_t>(L.grid) * kCandCap);
-  c.take<uint64_t>(static_cast<size_t>(L.grid) * cap);
-  c.take<uint32_t>(static_cast<size_t>(RG) * L.segs * L.seg_cap);
-  c.take<int32_t>(static_cast<size_t>(RG) * L.segs * L.seg_cap);
-  c.take<int32_t>(static_cast<size_t>(RG) * L.segs);
-  c.take<uint32_t>(static_cast<size_t>(RG) * L.segs);
-  c.take<uint64_t>(static_cast<size_t>(RG) * L.segs * L.seg_cap);
+  c.take<uint64_t>(static_cast<size_t>(L.grid) * comp);
+  c.take<uint32_t>(lists * L.list_cap);
+  c.take<int32_t>(lists * L.list_cap);
+  c.take<int32_t>(lists);
+  c.take<uint32_t>(lists);
+  c.take<uint64_t>(lists * L.list_cap);
   c.take<uint32_t>(static_cast<size_t>(RG) * bitmap_words(n_max));
   return c.used;
 }
@@ -1093,37 +1031,44 @@ size_t fused_ws_bytes(int RG, int n_max, int k, int B) {
 kvs_status fathom_scan_topk_launch(ScanParams p, void* ws, const int32_t* slot_map, int32_t* idx,
                                    int32_t* slots, int32_t* misses, cudaStream_t s,
                                    cudaEvent_t after_scan) {
+  if (p.B <= kPMaxB) {
+    // scores and 16-key group maxima from the byte-indexed scan, then the
+    // per-row top-k over them
+    WsCarver c(ws);
+    ScanParams q = p;
+    q.scores = c.take<float>(static_cast<size_t>(p.RG) * p.n_max);
+    q.gmax = c.take<float>(static_cast<size_t>(p.RG) * ((p.n_max + kPKeys - 1) / kPKeys));
+    uint32_t* bitmap = c.take<uint32_t>(static_cast<size_t>(p.RG) * bitmap_words(p.n_max));
+    kvs_status st = fathom_scan_lut_launch(q, s);
+    if (st != KVS_OK) return st;
+    if (after_scan) cudaEventRecord(after_scan, s);
+    cudaFuncSetAttribute(topk_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(kTkSmem));
+    topk_scores_kernel<<<p.RG, kTkThreads, kTkSmem, s>>>(q.scores, q.gmax, p.n, p.Gheads, p.n_max, p.k,
+                                                         bitmap, slot_map, idx, slots, misses);
+    return check_launch("decode_step(top-k over scores)");
+  }
   const Layout L = fused_layout(p.RG, p.n_max, p.k, p.B);
   if (L.grid <= 0) return KVS_OK;
-  if (L.segs > 64) return fail(KVS_EUNSUPPORTED, "decode_step: %d segments per row", L.segs);
+  if (L.segs * L.lists > 512) return fail(KVS_EUNSUPPORTED, "decode_step: %d segments per row", L.segs);
   p.chunks_per_row = L.cpr;
-  p.segs_per_row = L.segs;
-  p.seg_cap = L.seg_cap;
+  p.segs_per_row = L.segs * L.lists;
+  p.seg_cap = L.list_cap;
+  p.lists_per_seg = L.lists;
+  const size_t lists = static_cast<size_t>(p.RG) * p.segs_per_row;
+  const size_t comp = static_cast<size_t>(kCandCap > L.lists * L.list_cap ? kCandCap : L.lists * L.list_cap);
   WsCarver c(ws);
-  const size_t cap = static_cast<size_t>(kCandCap > L.seg_cap ? kCandCap : L.seg_cap);
   p.cbuf_key = c.take<uint32_t>(static_cast<size_t>(L.grid) * kCandCap);
   p.cbuf_idx = c.take<int32_t>(static_cast<size_t>(L.grid) * kCandCap);
-  p.cbuf_comp = c.take<uint64_t>(static_cast<size_t>(L.grid) * cap);
-  p.cand_key = c.take<uint32_t>(static_cast<size_t>(p.RG) * L.segs * L.seg_cap);
-  p.cand_idx = c.take<int32_t>(static_cast<size_t>(p.RG) * L.segs * L.seg_cap);
-  p.cand_count = c.take<int32_t>(static_cast<size_t>(p.RG) * L.segs);
-  p.cand_tau = c.take<uint32_t>(static_cast<size_t>(p.RG) * L.segs);
-  uint64_t* gscratch = c.take<uint64_t>(static_cast<size_t>(p.RG) * L.segs * L.seg_cap);
+  p.cbuf_comp = c.take<uint64_t>(static_cast<size_t>(L.grid) * comp);
+  p.cand_key = c.take<uint32_t>(lists * L.list_cap);
+  p.cand_idx = c.take<int32_t>(lists * L.list_cap);
+  p.cand_count = c.take<int32_t>(lists);
+  p.cand_tau = c.take<uint32_t>(lists);
+  uint64_t* gscratch = c.take<uint64_t>(lists * L.list_cap);
   uint32_t* bitmap = c.take<uint32_t>(static_cast<size_t>(p.RG) * bitmap_words(p.n_max));
-  kvs_status st;
-  if (p.B <= kPMaxB) {
-    p.nstage = prmt_nstages(p.B, kPFusedExtra);
-    if (p.nstage < 2) return fail(KVS_EUNSUPPORTED, "decode_step: no room for two stages at B=%d", p.B);
-    const size_t smem = prmt_smem_bytes(p.B, p.nstage, kPFusedExtra);
-    cudaFuncSetAttribute(fathom_scan_topk_prmt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(smem));
-    fathom_scan_topk_prmt_kernel<<<L.grid, kPThreadsStaged, smem, s>>>(p);
-    st = check_launch("decode_step(scan+topk, prmt)");
-  } else {
-    p.cand_tau = nullptr;
-    st = dispatch_schedule(p, FusedLaunch{p, L.grid, s});
-  }
-  if (st != KVS_OK) return st;
+  p.cand_tau = nullptr;  // this kernel keeps no per-list threshold
+  kvs_status st = dispatch_schedule(p, FusedLaunch{p, L.grid, s});
   if (after_scan) cudaEventRecord(after_scan, s);
   const size_t msmem = static_cast<size_t>(kMergeSmemEntries) * sizeof(uint64_t);
   cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
