@@ -45,14 +45,18 @@ WORKLOADS = {
     "tiny": dict(R=1, G=1, H=4, n=4096, B=92, k=256, S=512, miss=0.2),
 }
 METRIC = "index-scan keys/s + sparse decode layer-steps/s; achieved GB/s vs HBM peak"
+# the dominant kernel of a step with a plan of <= 144 planes: the byte-indexed
+# scan, which reads the plan's planes and writes every score and 16-key maximum
+SCAN_KERNEL = "fathom_scan_prmt (scan stage of the step)"
 
 # DRAM bytes (read + write) of one launch of the fused scan + top-k kernel, from
 # ncu captures of a smaller case of the same workload scaled to a full launch by
 # the keys processed (the capture and scaling are stated under profiles/);
 # None where no capture of the current kernel exists.
 TRAFFIC: dict = {
-    # R=8 capture: 96.61 MB read + 3.62 MB written per launch, x2 for R=16
-    ("qwen3-8b-128k", 92): 2 * (96_608_768 + 3_617_024),
+    # R=8 capture of fathom_scan_prmt_kernel: 96.55 MB read + 9.84 MB written
+    # per launch (the rest of its scores leave L2 later), x2 for R=16
+    ("qwen3-8b-128k", 92): 2 * (96_554_240 + 9_842_176),
 }
 
 
@@ -295,12 +299,13 @@ def run_ours(args, cfg, dist, rank, ws):
         "layer_steps_per_s": ws * 1e3 / ms_max,
         "achieved_gbs": algo["total"] * ws / (ms_max / 1e3) / 1e9,
         "miss_rate_measured": misses / (R * G * cfg["k"]),
-        "roofline": {"bound": "hbm", "kernel": "fathom_scan_topk (scan stage of the step)",
+        "roofline": {"bound": "hbm", "kernel": SCAN_KERNEL if cfg["B"] <= 144 else "fathom_scan_topk (scan stage of the step)",
                      "achieved": scan_bytes / (stages_ms["scan"] / 1e3) / 1e9, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": scan_bytes / (stages_ms["scan"] / 1e3) / 1e9 / peak,
                      "traffic": TRAFFIC.get((args.workload, cfg["B"])),
-                     "algorithmic_bytes": scan_bytes, "ms": stages_ms["scan"]},
+                     "algorithmic_bytes": scan_bytes, "ms": stages_ms["scan"],
+                     "bytes_moved": scan_bytes + algo["keys"] * (4 + 4 / 16) if cfg["B"] <= 144 else None},
         "stages_ms": stages_ms,
         "scan_only": {"kernel": "fathom_scan_lut (scores written to HBM)", "ms": scan_ms,
                       "achieved_gbs": scan_gbs, "frac": scan_gbs / peak},
