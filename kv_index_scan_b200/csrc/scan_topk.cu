@@ -1,27 +1,30 @@
-// scan_topk.cu -- a2 + a3 fused for decode_step: the Fathom scan keeps each
-// row's top-k candidates on chip instead of writing every score to HBM.
+// scan_topk.cu -- a2 + a3 for decode_step: the Fathom scan followed by the
+// per-row top-k, with the hot-buffer slot lookup of every selected key.
 //
 // Selection order is (score desc, index asc) ("XM-Sparse: Pushing the
 // Throughput Frontier of Sparse Attention with Netpreme X-Mem", modelled
 // study: 2,048 entries are picked per layer and step).
 //
-// Scan kernel (scan_core.cuh's pipeline, this epilogue): each block walks a
-// contiguous range of chunks; the part of one (request, KV head) row inside a
-// block is a "segment". Per segment the block appends to a buffer in L2 every
-// key whose score is at least a running threshold tau (all keys, until a
-// threshold exists), as (order-preserving score key, index). When the buffer
-// may not hold another chunk, two histogram passes over the held keys (bits
-// 31..21, then 20..10) find the cell holding the k-th largest key; tau becomes
-// that cell's lower edge and every held key below it is dropped. The held set
-// always contains the segment's top-k (at least k keys are >= tau), so nothing
-// of the answer is ever lost; it is a superset, trimmed again at the segment's
-// end (and cut exactly to k only if it would still be too large).
+// Plans of at most 144 planes: the byte-indexed scan writes every score and
+// the maximum of every 16 keys; topk_scores_kernel (below) selects from them,
+// one block per row, reading only the groups whose maximum can reach the
+// row's k-th score.
 //
-// Merge kernel: one block per row gathers its segments' candidates as
-// distinct 53-bit composites (score key << 21 | (2^21 - 1 - index)), selects
-// exactly the k largest (radix passes), emits their indices in ascending order
-// through a bitmap over the row, and looks every selected key up in the
-// hot-buffer slot map (slots; misses = the number absent from the hot buffer).
+// Larger plans: the group-table scan keeps each row's candidates on chip.
+// Each block walks a contiguous range of chunks; the part of one (request, KV
+// head) row inside a block is a "segment". Per segment the block appends to a
+// buffer in L2 every key whose score is at least a running threshold tau (all
+// keys, until a threshold exists), as (order-preserving score key, index).
+// When the buffer may not hold another chunk, two histogram passes over the
+// held keys (bits 31..21, then 20..10) find the cell holding the k-th largest
+// key; tau becomes that cell's lower edge and every held key below it is
+// dropped. The held set always contains the segment's top-k (at least k keys
+// are >= tau), so nothing of the answer is ever lost. A merge kernel, one
+// block per row, gathers the segments' candidates as distinct 53-bit
+// composites (score key << 21 | (2^21 - 1 - index)), selects exactly the k
+// largest (radix passes), emits their indices in ascending order through a
+// bitmap over the row, and looks every selected key up in the hot-buffer slot
+// map (slots; misses = the number absent from the hot buffer).
 #include "internal.cuh"
 #include "scan_core.cuh"
 #include "scan_prmt.cuh"
@@ -608,25 +611,38 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(
 // (the byte-indexed scan writes both). One block of 1,024 threads per row.
 //  A. T = (a lower bound of) the kk-th largest group maximum: each group
 //     maximum is a distinct key, so at least kk keys are >= T and the row's
-//     kk-th largest score is >= T. Groups whose maximum is below T hold no
-//     selected key and are never read again (about a quarter of the groups
-//     remain for Gaussian-like scores).
-//  B. Radix select (11/11/10 bits of the order-preserving key) over the keys
-//     >= T of the remaining groups: either a whole key cell holds the last
-//     selected ranks (select every key >= its lower edge: exactly kk keys), or
-//     the exact kk-th largest key K* (select the keys > K*, and of the keys
-//     equal to K* the lowest indices).
-//  C. The selected keys are marked in a bitmap over the row, ties by index
-//     order (groups are visited in index order in rounds of 1,024 with one
-//     block-wide scan per round), and emitted in ascending order with the
-//     slot of each and the row's miss count.
+//     kk-th largest score is >= T. The maxima are kept as 16-bit key prefixes,
+//     selected in 12-bit digits from the highest bit in which they differ
+//     (one digit when they span less than 2^12 prefixes).
+//     Groups whose maximum is below T hold no selected key and are never read
+//     (about a quarter of the groups remain for Gaussian-like scores).
+//  B. The remaining groups are listed in index order (8 per thread, one
+//     block-wide scan per 8,192 groups).
+//  C. Each warp takes a contiguous slice of that list, four lanes per group
+//     (one 16-byte load each, so a warp's load touches 8 groups' lines), and
+//     appends its keys >= T with their indices, in index order, to a list of
+//     its own; the warps' lists in warp order are the row's candidates in
+//     index order.
+//  D. Radix select over the candidates in digits of up to 12 bits, from the
+//     highest bit in which the smallest and the largest candidate differ:
+//     either a whole key cell holds the last selected ranks (select every key
+//     >= its lower edge: exactly kk keys), or the exact kk-th largest key K*
+//     (select the keys > K*, and of the keys equal to K* the lowest indices).
+//  E. Each warp emits its selected keys at their ranks in index order (one
+//     block-wide exchange of the warps' counts), with the slot of each; the
+//     row's miss count closes the kernel.
+// Rows longer than 65,536 groups, or whose candidates overflow the on-chip
+// lists, take the same selection over global memory with a bitmap.
 constexpr int kTkThreads = 1024;
+constexpr int kTkWarps = kTkThreads / 32;
+constexpr int kTkBins = 4096;
 
 struct TkState {
   int wsum[32], res[2];
   uint32_t prefix, mask;
   int krem, done, gt;
-  int tie_base;
+  int wcnt[32], ws[32], wt[32];
+  uint32_t wmin[32], wmax[32];
   int miss_warp[32];
 };
 
@@ -673,11 +689,49 @@ __device__ uint32_t radix_kth_key(Each&& each, int kk, unsigned* hist, TkState* 
   return st->prefix;
 }
 
+// The same select when every key agrees with `prefix` on the bits above `top`:
+// digits of up to 12 bits from bit `top` down.
+template <typename Each>
+__device__ uint32_t radix_select_from(Each&& each, int top, uint32_t prefix, int kk, unsigned* hist,
+                                      TkState* st, bool* whole, int* gt) {
+  const int t = threadIdx.x;
+  uint32_t mask = top >= 31 ? 0u : ~((2u << top) - 1u);
+  int krem = kk, above = 0;
+  for (;;) {
+    const int width = min(12, top + 1);
+    const int shift = top + 1 - width;
+    const uint32_t dmask = (1u << width) - 1u;
+    const int nb = 1 << width;
+    for (int b = t; b < nb; b += kTkThreads) hist[b] = 0;
+    __syncthreads();
+    each([&](uint32_t key) {
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+    });
+    __syncthreads();
+    find_bin_from_top(hist, nb, krem, st->wsum, st->res, t, kTkThreads, [] { __syncthreads(); });
+    const int bin = st->res[0];
+    const int ab = st->res[1];
+    const int inbin = static_cast<int>(hist[bin]);
+    prefix |= static_cast<uint32_t>(bin) << shift;
+    mask |= dmask << shift;
+    krem -= ab;
+    above += ab;
+    const int done = krem == inbin ? 1 : (shift == 0 ? 2 : 0);
+    __syncthreads();  // hist[bin] and res are read before the next pass rewrites them
+    if (done) {
+      *whole = done == 1;
+      *gt = above;
+      return prefix;
+    }
+    top = shift - 1;
+  }
+}
+
 constexpr int kTkMaxGroups = 65536;  // group maxima kept in shared memory (16-bit prefixes)
-constexpr int kTkCandGroups = 6144;  // candidate groups, and candidate keys, on chip
-constexpr int kTkCandKeys = 6144;
-constexpr size_t kTkSmem = kTkMaxGroups * sizeof(uint16_t) + kTkCandGroups * sizeof(int) +
-                           kTkCandKeys * sizeof(uint2);
+constexpr int kTkCandGroups = 8192;  // candidate groups on chip
+// per-warp candidate lists (key, index), over the maxima once those are read
+constexpr int kTkWarpKeys = static_cast<int>(kTkMaxGroups * sizeof(uint16_t) / (kTkWarps * sizeof(uint2)));
+constexpr size_t kTkSmem = kTkMaxGroups * sizeof(uint16_t) + kTkCandGroups * sizeof(int);
 
 // Block-wide exclusive prefix of c over the threads (in thread order); returns
 // it and the block total.
@@ -701,16 +755,18 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(
     const float* __restrict__ scores, const float* __restrict__ gmax, const int32_t* __restrict__ n,
     int Gheads, int n_max, int k, uint32_t* __restrict__ bitmap, const int32_t* __restrict__ slot_map,
     int32_t* __restrict__ idx, int32_t* __restrict__ slots, int32_t* __restrict__ misses) {
-  __shared__ unsigned hist[2048];
+  __shared__ unsigned hist[kTkBins];
   __shared__ TkState st;
   extern __shared__ __align__(16) unsigned char tk_smem[];
-  uint16_t* gk = reinterpret_cast<uint16_t*>(tk_smem);                      // [kTkMaxGroups]
+  uint16_t* gk = reinterpret_cast<uint16_t*>(tk_smem);                          // [kTkMaxGroups]
+  uint2* lists = reinterpret_cast<uint2*>(tk_smem);                              // [kTkWarps][kTkWarpKeys]
   int* cg = reinterpret_cast<int*>(tk_smem + kTkMaxGroups * sizeof(uint16_t));  // [kTkCandGroups]
-  uint2* ck = reinterpret_cast<uint2*>(cg + kTkCandGroups);                 // [kTkCandKeys] (key, index)
   constexpr int NG = 16;  // keys per group
+  constexpr unsigned FULL = 0xFFFFFFFFu;
   const float ninf = -__int_as_float(0x7f800000);
   const int u = blockIdx.x;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const unsigned lt = (1u << lane) - 1u;
   const int nr = min(n[u / Gheads], n_max);
   const int kk = min(k, nr);
   const int ldg = (n_max + NG - 1) / NG;
@@ -718,211 +774,316 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(
   const float* sc = scores + static_cast<size_t>(u) * n_max;
   const float* gm = gmax + static_cast<size_t>(u) * ldg;
   const bool vec = (n_max & 3) == 0;
-  const int words = bitmap_words(n_max);
-  uint32_t* bm = bitmap + static_cast<size_t>(u) * words;
-  for (int w = 4 * t; w < words; w += 4 * kTkThreads)
-    *reinterpret_cast<uint4*>(bm + w) = make_uint4(0u, 0u, 0u, 0u);
+  int32_t* irow = idx + static_cast<size_t>(u) * k;
+  int32_t* srow = slots ? slots + static_cast<size_t>(u) * k : nullptr;
+  const int32_t* smap = slot_map ? slot_map + static_cast<size_t>(u) * n_max : nullptr;
 
-  // the 16 scores of group g (invalid keys: -inf, written by the scan)
-  auto load_group = [&](int g, float (&v)[NG]) {
-    const float* src = sc + static_cast<size_t>(g) * NG;
-    if (vec && g * NG + NG <= n_max) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 f = __ldg(reinterpret_cast<const float4*>(src) + q);
-        v[4 * q] = f.x;
-        v[4 * q + 1] = f.y;
-        v[4 * q + 2] = f.z;
-        v[4 * q + 3] = f.w;
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < NG; ++j) v[j] = g * NG + j < n_max ? __ldg(src + j) : ninf;
-    }
-  };
-
-  bool whole = true;
-  int gt = 0;
-  uint32_t key_cut = 0u;
-  int nck = -1;  // keys >= T on chip (-1: too many, the rows' scores are read again)
+  bool onchip = kk > 0 && m <= kTkMaxGroups;
   uint32_t T = 0u;
-  if (kk > 0 && m <= kTkMaxGroups) {
-    // A. the group maxima on chip as 16-bit key prefixes; T from them (at
-    // least kk maxima have a prefix >= T's, so at least kk keys are >= T)
-#pragma unroll 4
-    for (int g = t; g < m; g += kTkThreads) gk[g] = static_cast<uint16_t>(ordered_key(__ldg(gm + g)) >> 16);
+  int my_miss = 0;
+  if (onchip) {
+    // A. maxima as 16-bit prefixes, with their range; T
+    uint32_t pmin = 0xFFFFu, pmax = 0u;
+#pragma unroll 8
+    for (int g = t; g < m; g += kTkThreads) {
+      const uint32_t pfx = ordered_key(__ldg(gm + g)) >> 16;
+      gk[g] = static_cast<uint16_t>(pfx);
+      pmin = min(pmin, pfx);
+      pmax = max(pmax, pfx);
+    }
+    pmin = __reduce_min_sync(FULL, pmin);
+    pmax = __reduce_max_sync(FULL, pmax);
+    if (lane == 0) {
+      st.wmin[warp] = pmin;
+      st.wmax[warp] = pmax;
+    }
     __syncthreads();
     if (kk <= m) {
+      const uint32_t lo = __reduce_min_sync(FULL, st.wmin[lane]);
+      const uint32_t x = lo ^ __reduce_max_sync(FULL, st.wmax[lane]);
+      const int top = x ? 31 - __clz(x) : 0;
       bool wh;
       int g0;
-      T = radix_kth_key([&](auto visit) {
-            for (int g = t; g < m; g += kTkThreads) visit(static_cast<uint32_t>(gk[g]) << 16);
-          }, kk, hist, &st, &wh, &g0) & 0xFFFF0000u;
+      T = radix_select_from([&](auto visit) {
+            for (int g = t; g < m; g += kTkThreads) visit(static_cast<uint32_t>(gk[g]));
+          }, top, lo & ~((2u << top) - 1u), kk, hist, &st, &wh, &g0) << 16;
     }
-    // candidate groups in index order
+    // B. candidate groups in index order
+    const uint32_t Tp = T >> 16;
     int ncg = 0;
-    for (int r0 = 0; r0 < m; r0 += kTkThreads) {
-      const int g = r0 + t;
-      const int c = g < m && (static_cast<uint32_t>(gk[g]) << 16) >= T ? 1 : 0;
+    for (int r0 = 0; r0 < m; r0 += 8 * kTkThreads) {
+      const int g0 = r0 + 8 * t;
+      uint32_t flags = 0u;
+      if (g0 < m) {
+        const uint4 w = *reinterpret_cast<const uint4*>(gk + g0);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t pfx = (ww[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+          if (g0 + j < m && pfx >= Tp) flags |= 1u << j;
+        }
+      }
       int tot;
-      const int pos = block_excl_scan(c, &st, &tot);
-      if (c && ncg + pos < kTkCandGroups) cg[ncg + pos] = g;
+      int q = ncg + block_excl_scan(__popc(flags), &st, &tot);
+      if (q + __popc(flags) <= kTkCandGroups) {
+        while (flags) {
+          const int j = __ffs(flags) - 1;
+          flags &= flags - 1u;
+          cg[q++] = g0 + j;
+        }
+      }
       ncg += tot;
     }
-    if (ncg <= kTkCandGroups) {
-      // keys >= T of the candidate groups, in index order (the groups' scores
-      // are loaded in one round per 1,024 groups)
-      nck = 0;
-      for (int r0 = 0; r0 < ncg; r0 += kTkThreads) {
-        const int e = r0 + t;
-        float v[NG];
-        uint32_t pass = 0u;
-        int g = 0;
-        if (e < ncg) {
-          g = cg[e];
-          load_group(g, v);
+    onchip = ncg <= kTkCandGroups;
+    if (onchip) {
+      __syncthreads();  // cg is complete; the maxima are no longer read
+      // C. this warp's slice of the candidate groups, four lanes per group
+      const int per_w = (ncg + kTkWarps - 1) / kTkWarps;
+      const int e_beg = min(ncg, warp * per_w), e_end = min(ncg, e_beg + per_w);
+      uint2* wl = lists + warp * kTkWarpKeys;
+      const int sub = lane >> 2, qtr = lane & 3;
+      int wc = 0;
+      bool ovf = false;
+      uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+      // four iterations' loads in flight per warp
+      constexpr int kU = 4;
+      const int niter = (e_end - e_beg + 7) >> 3;
+      for (int it0 = 0; it0 < niter && !ovf; it0 += kU) {
+        float4 f[kU];
+        int base[kU];
 #pragma unroll
-          for (int j = 0; j < NG; ++j)
-            if (g * NG + j < nr && ordered_key(v[j]) >= T) pass |= 1u << j;
-        }
-        int tot;
-        int pos = nck + block_excl_scan(__popc(pass), &st, &tot);
-        if (nck + tot <= kTkCandKeys) {
-          while (pass) {
-            const int j = __ffs(pass) - 1;
-            pass &= pass - 1u;
-            ck[pos++] = make_uint2(ordered_key(v[j]), static_cast<uint32_t>(g * NG + j));
+        for (int a = 0; a < kU; ++a) {
+          const int e = e_beg + 8 * (it0 + a) + sub;
+          base[a] = -1;
+          f[a] = make_float4(ninf, ninf, ninf, ninf);
+          if (it0 + a < niter && e < e_end) {
+            base[a] = cg[e] * NG + 4 * qtr;
+            if (vec && base[a] + 4 <= n_max) {
+              f[a] = __ldg(reinterpret_cast<const float4*>(sc + base[a]));
+            } else {
+              const float* s0 = sc + base[a];
+              f[a].x = base[a] < n_max ? __ldg(s0) : ninf;
+              f[a].y = base[a] + 1 < n_max ? __ldg(s0 + 1) : ninf;
+              f[a].z = base[a] + 2 < n_max ? __ldg(s0 + 2) : ninf;
+              f[a].w = base[a] + 3 < n_max ? __ldg(s0 + 3) : ninf;
+            }
           }
         }
-        nck += tot;
+#pragma unroll
+        for (int a = 0; a < kU; ++a) {
+          if (it0 + a >= niter) break;
+          const float v[4] = {f[a].x, f[a].y, f[a].z, f[a].w};
+          uint32_t pass = 0u;
+          if (base[a] >= 0) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if (base[a] + j < nr && ordered_key(v[j]) >= T) pass |= 1u << j;
+          }
+          const int c = __popc(pass);
+          const unsigned b0 = __ballot_sync(FULL, c & 1), b1 = __ballot_sync(FULL, c & 2),
+                         b2 = __ballot_sync(FULL, c & 4);
+          const int tot = __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2);
+          if (wc + tot > kTkWarpKeys) {
+            ovf = true;
+            break;
+          }
+          int q = wc + __popc(b0 & lt) + 2 * __popc(b1 & lt) + 4 * __popc(b2 & lt);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if ((pass >> j) & 1u) {
+              const uint32_t key = ordered_key(v[j]);
+              wl[q++] = make_uint2(key, static_cast<uint32_t>(base[a] + j));
+              kmin = min(kmin, key);
+              kmax = max(kmax, key);
+            }
+          }
+          wc += tot;
+        }
       }
-      if (nck > kTkCandKeys) nck = -1;
+      kmin = __reduce_min_sync(FULL, kmin);
+      kmax = __reduce_max_sync(FULL, kmax);
+      if (lane == 0) {
+        st.wcnt[warp] = ovf ? -1 : wc;
+        st.wmin[warp] = kmin;
+        st.wmax[warp] = kmax;
+      }
+      __syncthreads();
+      onchip = !__any_sync(FULL, st.wcnt[lane] < 0);
+      if (onchip) {
+        // D. the kk-th largest candidate key
+        const uint32_t lo = __reduce_min_sync(FULL, st.wmin[lane]);
+        const uint32_t hi = __reduce_max_sync(FULL, st.wmax[lane]);
+        const uint32_t x = lo ^ hi;
+        const int top = x ? 31 - __clz(x) : 0;
+        const uint32_t upper = top >= 31 ? 0u : ~((2u << top) - 1u);
+        bool whole;
+        int gt;
+        const uint32_t cut = radix_select_from([&](auto visit) {
+              for (int i = lane; i < wc; i += 32) visit(wl[i].x);
+            }, top, lo & upper, kk, hist, &st, &whole, &gt);
+        // E. ranks in index order: keys above the cut, then the first `need` ties
+        const int need = whole ? 0 : kk - gt;
+        int ns = 0, nt = 0;
+        for (int i = lane; i < wc; i += 32) {
+          const uint32_t key = wl[i].x;
+          ns += (whole ? key >= cut : key > cut) ? 1 : 0;
+          nt += (!whole && key == cut) ? 1 : 0;
+        }
+        ns = __reduce_add_sync(FULL, ns);
+        nt = __reduce_add_sync(FULL, nt);
+        if (lane == 0) {
+          st.ws[warp] = ns;
+          st.wt[warp] = nt;
+        }
+        __syncthreads();
+        int s_run = __reduce_add_sync(FULL, lane < warp ? st.ws[lane] : 0);
+        int t_run = __reduce_add_sync(FULL, lane < warp ? st.wt[lane] : 0);
+        for (int i0 = 0; i0 < wc; i0 += 32) {
+          const int i = i0 + lane;
+          const uint2 c = i < wc ? wl[i] : make_uint2(0u, 0u);
+          const bool strict = i < wc && (whole ? c.x >= cut : c.x > cut);
+          const bool tie = i < wc && !whole && c.x == cut;
+          const unsigned bs = __ballot_sync(FULL, strict), bt = __ballot_sync(FULL, tie);
+          const int sb = s_run + __popc(bs & lt), tb = t_run + __popc(bt & lt);
+          const int pos = sb + min(tb, need);
+          if ((strict || (tie && tb < need)) && pos < kk) {
+            const int ix = static_cast<int>(c.y);
+            irow[pos] = ix;
+            const int sl = smap ? smap[ix] : -1;
+            my_miss += sl < 0 ? 1 : 0;
+            if (srow) srow[pos] = sl;
+          }
+          s_run += __popc(bs);
+          t_run += __popc(bt);
+        }
+        for (int j = kk + t; j < k; j += kTkThreads) {
+          irow[j] = -1;
+          if (srow) srow[j] = -2;
+        }
+      }
+    }
+  }
+  if (!onchip) {
+    // too many candidates for the chip (or no row at all): the same selection
+    // over the rows' scores in global memory (groups whose maximum is below T
+    // are skipped), emitted through a bitmap over the row
+    const int words = bitmap_words(n_max);
+    uint32_t* bm = bitmap + static_cast<size_t>(u) * words;
+    for (int w = 4 * t; w < words; w += 4 * kTkThreads)
+      *reinterpret_cast<uint4*>(bm + w) = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+    auto load_group = [&](int g, float (&v)[NG]) {
+      const float* src = sc + static_cast<size_t>(g) * NG;
+      if (vec && g * NG + NG <= n_max) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 f = __ldg(reinterpret_cast<const float4*>(src) + q);
+          v[4 * q] = f.x;
+          v[4 * q + 1] = f.y;
+          v[4 * q + 2] = f.z;
+          v[4 * q + 3] = f.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < NG; ++j) v[j] = g * NG + j < n_max ? __ldg(src + j) : ninf;
+      }
+    };
+    if (kk > 0) {
+      bool whole;
+      int gt;
+      const uint32_t key_cut = radix_kth_key([&](auto visit) {
+            for (int g = t; g < m; g += kTkThreads) {
+              if (ordered_key(__ldg(gm + g)) < T) continue;
+              float v[NG];
+              load_group(g, v);
+#pragma unroll
+              for (int j = 0; j < NG; ++j)
+                if (g * NG + j < nr) {
+                  const uint32_t key = ordered_key(v[j]);
+                  if (key >= T) visit(key);
+                }
+            }
+          }, kk, hist, &st, &whole, &gt);
+      const int need = whole ? 0 : kk - gt;
+      int tie_base = 0;
+      for (int r0 = 0; r0 < m; r0 += kTkThreads) {
+        const int g = r0 + t;
+        uint32_t sel = 0u, tie = 0u;
+        if (g < m && ordered_key(__ldg(gm + g)) >= key_cut) {
+          float v[NG];
+          load_group(g, v);
+#pragma unroll
+          for (int j = 0; j < NG; ++j) {
+            if (g * NG + j >= nr) continue;
+            const uint32_t key = ordered_key(v[j]);
+            if (whole ? key >= key_cut : key > key_cut) sel |= 1u << j;
+            else if (!whole && key == key_cut) tie |= 1u << j;
+          }
+        }
+        if (!whole) {
+          int tot;
+          int rank = tie_base + block_excl_scan(__popc(tie), &st, &tot);
+          while (tie) {
+            const int j = __ffs(tie) - 1;
+            tie &= tie - 1u;
+            if (rank < need) sel |= 1u << j;
+            ++rank;
+          }
+          tie_base += tot;
+        }
+        if (sel) atomicOr(bm + (g >> 1), (g & 1) ? (sel << 16) : sel);
+      }
     }
     __syncthreads();
-  }
-
-  if (kk > 0 && nck >= 0) {
-    // B. on chip: the kk-th largest candidate key
-    key_cut = radix_kth_key([&](auto visit) {
-                for (int e = t; e < nck; e += kTkThreads) visit(ck[e].x);
-              }, kk, hist, &st, &whole, &gt);
-    // C. mark the selected keys; ties by index (the list is in index order)
-    const int need = whole ? 0 : kk - gt;
-    int tie_base = 0;
-    for (int r0 = 0; r0 < nck; r0 += kTkThreads) {
-      const int e = r0 + t;
-      uint2 c = make_uint2(0u, 0u);
-      bool sel = false, tie = false;
-      if (e < nck) {
-        c = ck[e];
-        sel = whole ? c.x >= key_cut : c.x > key_cut;
-        tie = !whole && c.x == key_cut;
-      }
-      if (!whole) {
-        int tot;
-        const int rank = tie_base + block_excl_scan(tie ? 1 : 0, &st, &tot);
-        if (tie && rank < need) sel = true;
-        tie_base += tot;
-      }
-      if (sel) atomicOr(bm + (c.y >> 5), 1u << (c.y & 31));
+    // ascending emission: thread t owns words [t * wpt, (t + 1) * wpt)
+    const int wpt = ((words + kTkThreads - 1) / kTkThreads + 3) & ~3;
+    const int w_beg = min(words, t * wpt), w_end = min(words, w_beg + wpt);
+    int cnt = 0;
+    for (int w = w_beg; w < w_end; w += 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(bm + w);
+      cnt += __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
     }
-  } else if (kk > 0) {
-    // too many candidates for the chip: the same selection over the rows'
-    // scores in global memory (groups whose maximum is below T are skipped)
-    key_cut = radix_kth_key([&](auto visit) {
-                for (int g = t; g < m; g += kTkThreads) {
-                  if (ordered_key(__ldg(gm + g)) < T) continue;
-                  float v[NG];
-                  load_group(g, v);
+    int incl = cnt;
 #pragma unroll
-                  for (int j = 0; j < NG; ++j)
-                    if (g * NG + j < nr) {
-                      const uint32_t key = ordered_key(v[j]);
-                      if (key >= T) visit(key);
-                    }
-                }
-              }, kk, hist, &st, &whole, &gt);
-    const int need = whole ? 0 : kk - gt;
-    int tie_base = 0;
-    for (int r0 = 0; r0 < m; r0 += kTkThreads) {
-      const int g = r0 + t;
-      uint32_t sel = 0u, tie = 0u;
-      if (g < m && ordered_key(__ldg(gm + g)) >= key_cut) {
-        float v[NG];
-        load_group(g, v);
-#pragma unroll
-        for (int j = 0; j < NG; ++j) {
-          if (g * NG + j >= nr) continue;
-          const uint32_t key = ordered_key(v[j]);
-          if (whole ? key >= key_cut : key > key_cut) sel |= 1u << j;
-          else if (!whole && key == key_cut) tie |= 1u << j;
-        }
+    for (int d = 1; d < 32; d <<= 1) {
+      const int o = __shfl_up_sync(FULL, incl, d);
+      if (lane >= d) incl += o;
+    }
+    if (lane == 31) st.wsum[warp] = incl;
+    __syncthreads();
+    const int before = __reduce_add_sync(FULL, lane < warp ? st.wsum[lane] : 0);
+    int pos = before + incl - cnt;
+    for (int w = w_beg; w < w_end && cnt > 0; ++w) {
+      uint32_t bits = bm[w];
+      while (bits) {
+        const int bpos = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        if (pos < k) irow[pos] = 32 * w + bpos;
+        ++pos;
       }
-      if (!whole) {
-        int tot;
-        int rank = tie_base + block_excl_scan(__popc(tie), &st, &tot);
-        while (tie) {
-          const int j = __ffs(tie) - 1;
-          tie &= tie - 1u;
-          if (rank < need) sel |= 1u << j;
-          ++rank;
-        }
-        tie_base += tot;
+    }
+    __syncthreads();
+    const int chosen_total = min(__reduce_add_sync(FULL, st.wsum[lane]), kk);
+    for (int j = t; j < k; j += kTkThreads) {
+      int i = -1;
+      if (j < chosen_total)
+        i = irow[j];
+      else
+        irow[j] = -1;
+      int sl = -2;
+      if (i >= 0) {
+        sl = smap ? smap[i] : -1;
+        my_miss += sl < 0 ? 1 : 0;
       }
-      if (sel) atomicOr(bm + (g >> 1), (g & 1) ? (sel << 16) : sel);
+      if (srow) srow[j] = sl;
     }
   }
-  __syncthreads();
-  // ascending emission: thread t owns words [t * wpt, (t + 1) * wpt)
-  const int wpt = ((words + kTkThreads - 1) / kTkThreads + 3) & ~3;
-  const int w_beg = min(words, t * wpt), w_end = min(words, w_beg + wpt);
-  int cnt = 0;
-  for (int w = w_beg; w < w_end; w += 4) {
-    const uint4 v = *reinterpret_cast<const uint4*>(bm + w);
-    cnt += __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
-  }
-  int incl = cnt;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-    if (lane >= d) incl += o;
-  }
-  if (lane == 31) st.wsum[warp] = incl;
-  __syncthreads();
-  const int before = __reduce_add_sync(0xFFFFFFFFu, lane < warp ? st.wsum[lane] : 0);
-  int pos = before + incl - cnt;
-  int32_t* irow = idx + static_cast<size_t>(u) * k;
-  for (int w = w_beg; w < w_end && cnt > 0; ++w) {
-    uint32_t bits = bm[w];
-    while (bits) {
-      const int bpos = __ffs(bits) - 1;
-      bits &= bits - 1u;
-      if (pos < k) irow[pos] = 32 * w + bpos;
-      ++pos;
-    }
-  }
-  __syncthreads();
-  const int chosen_total = min(__reduce_add_sync(0xFFFFFFFFu, st.wsum[lane]), kk);
-  int my_miss = 0;
-  for (int j = t; j < k; j += kTkThreads) {
-    int i = -1;
-    if (j < chosen_total)
-      i = irow[j];
-    else
-      irow[j] = -1;
-    int sl = -2;
-    if (i >= 0) {
-      sl = slot_map ? slot_map[static_cast<size_t>(u) * n_max + i] : -1;
-      my_miss += sl < 0 ? 1 : 0;
-    }
-    if (slots) slots[static_cast<size_t>(u) * k + j] = sl;
-  }
-  const int wm = __reduce_add_sync(0xFFFFFFFFu, my_miss);
+  const int wm = __reduce_add_sync(FULL, my_miss);
   if (lane == 0) st.miss_warp[warp] = wm;
   __syncthreads();
   if (t == 0 && misses) {
     int mm = 0;
-    for (int e = 0; e < kTkThreads / 32; ++e) mm += st.miss_warp[e];
+    for (int e = 0; e < kTkWarps; ++e) mm += st.miss_warp[e];
     misses[u] = mm;
   }
 }
