@@ -15,8 +15,8 @@
 //  * Each warp streams its own 16-row tiles through a three-stage ring in
 //    shared memory with cp.async (16-byte copies, zero fill for padding rows,
 //    chunk c of row r stored at c ^ (r & 7) so that ldmatrix reads are
-//    conflict-free). The row locations of a tile are fetched one tile ahead of
-//    its copies, and its copies two tiles ahead of its arithmetic.
+//    conflict-free). The row locations of a tile are fetched four tiles ahead
+//    of its copies, and its copies two tiles ahead of its arithmetic.
 //  * Logits: S^T[heads][rows] = Q K^T with mma.m16n8k16 (bf16 inputs, f32
 //    accumulation). The 16 MMA rows hold q split in two bf16 parts, q_hi in
 //    rows 0..7 and q - q_hi in rows 8..15, so one MMA carries q to ~16 bits
@@ -98,6 +98,12 @@ __device__ __forceinline__ int row_code(const RowSrc& src, int u, int j) {
   }
   const int32_t* irow =
       src.idx + (src.idx_shared ? static_cast<size_t>(u / src.G) : static_cast<size_t>(u)) * src.k;
+  if (src.mode == kRowsSlot && src.slots) {
+    // both loads issued together (the slot of a padding entry is not used)
+    const int i = __ldg(irow + j);
+    const int sl = __ldg(src.slots + static_cast<size_t>(u) * src.k + j);
+    return i < 0 ? -1 : (sl >= 0 ? -2 - sl : i);
+  }
   const int i = irow[j];
   if (i < 0) return -1;
   if (src.mode == kRowsSlot) {
@@ -200,15 +206,24 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnBlocksPerSM) sparse_attn_ke
     for (int e = 0; e < 4; ++e) o[d][e] = 0.f;
   float m_run = ninf, l_run = 0.f;  // of head g, shared by the four lanes of group g
 
-  // prologue: tiles 0 and 1 in flight, the codes of tile 2 on their way
+  // prologue: tiles 0 and 1 in flight, the codes of tiles 2..5 on their way
+  // (row locations are fetched four tiles ahead of their copies)
+  // The codes of tile t live in register c[t % 4] (the loop is unrolled by 4
+  // so that each stays in place until used: moving a register whose load is
+  // still in flight would wait for it).
   unsigned vm0 = issue(0, fetch_code(0), 0);
   unsigned vm1 = issue(1, fetch_code(1), 1);
-  int code_next = fetch_code(2);
+  int c0 = fetch_code(4), c1 = fetch_code(5), c2 = fetch_code(2), c3 = fetch_code(3);
 
-  for (int i = 0; i < ntiles; ++i) {
+  for (int i0 = 0; i0 < ntiles; i0 += 4)
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int i = i0 + a;
+    if (i >= ntiles) break;
+    int& code_cur = a == 0 ? c2 : (a == 1 ? c3 : (a == 2 ? c0 : c1));  // tile i + 2's
     const int st = i % kAttnStages;
-    const unsigned vm2 = issue(i + 2, code_next, (i + 2) % kAttnStages);
-    code_next = fetch_code(i + 3);
+    const unsigned vm2 = issue(i + 2, code_cur, (i + 2) % kAttnStages);
+    code_cur = fetch_code(i + 6);
     cp_async_wait<kAttnStages - 1>();
     __syncwarp();
     const uint32_t kst = ring + st * kStageBytes;

@@ -11,9 +11,9 @@
 // (value desc, c asc, j asc). Every event gets a distinct 64-bit key -- the bit
 // pattern of the exact double w_c 4^-j (an f32 widened to fp64 has 29 zero low
 // mantissa bits) with 511 - (4c + j) in the low bits -- and the events whose
-// keys are among the B largest are taken: a bitonic sort of the 512 keys in
-// shared memory (descending), the first B of it marked. One 512-thread block
-// per (r, g).
+// keys are among the B largest are taken: a bitonic sort of the 512 keys
+// (descending; warp shuffles for partners closer than 32, shared memory
+// beyond), the first B of it marked. One 512-thread block per (r, g).
 #include "internal.cuh"
 
 namespace kvs {
@@ -28,7 +28,7 @@ __global__ void __launch_bounds__(512) plan_bits_kernel(
   const int u = blockIdx.x;
   const int tid = threadIdx.x;
   __shared__ float qb[kD], wv[kD];
-  __shared__ unsigned long long key[4 * kD];
+  __shared__ unsigned long long kbuf[2][4 * kD];
   __shared__ int tcount[kD], start[kD];
   __shared__ unsigned char took[4 * kD];
   __shared__ float cterm[kD];
@@ -41,33 +41,35 @@ __global__ void __launch_bounds__(512) plan_bits_kernel(
   }
   __syncthreads();
   const int c = tid >> 2, j = tid & 3;
+  unsigned long long x;
   {
     const double scale = j == 0 ? 1.0 : j == 1 ? 0.25 : j == 2 ? 0.0625 : 0.015625;
     double v = __dmul_rn(static_cast<double>(wv[c]), scale);
     v = v > 0.0 ? v : 0.0;  // -0 -> +0 (weights are non-negative)
-    key[tid] = static_cast<unsigned long long>(__double_as_longlong(v)) |
-               static_cast<unsigned long long>(511 - tid);
+    x = static_cast<unsigned long long>(__double_as_longlong(v)) | static_cast<unsigned long long>(511 - tid);
   }
   took[tid] = 0;
-  __syncthreads();
-  // bitonic sort, descending: thread tid < 256 owns one compare-exchange pair
-  // per stage
+  // bitonic sort, descending, one key per thread: the partner at distance
+  // `stride` is read by warp shuffle below 32 and through shared memory (two
+  // buffers in turn, one barrier per stage) above
+  int buf = 0;
   for (int size = 2; size <= 4 * kD; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      if (tid < 2 * kD) {
-        const int lo = 2 * tid - (tid & (stride - 1));
-        const int hi = lo + stride;
-        const bool desc = (lo & size) == 0;
-        const unsigned long long a = key[lo], b = key[hi];
-        if ((a < b) == desc) {
-          key[lo] = b;
-          key[hi] = a;
-        }
+      unsigned long long y;
+      if (stride >= 32) {
+        kbuf[buf][tid] = x;
+        __syncthreads();
+        y = kbuf[buf][tid ^ stride];
+        buf ^= 1;
+      } else {
+        y = __shfl_xor_sync(0xFFFFFFFFu, x, stride);
       }
-      __syncthreads();
+      const bool keep_max = ((tid & size) == 0) == ((tid & stride) == 0);
+      x = keep_max ? (x > y ? x : y) : (x < y ? x : y);
     }
   }
-  if (tid < B) took[511 - static_cast<int>(key[tid] & 511ull)] = 1;
+  __syncthreads();  // took[] cleared by every thread
+  if (tid < B) took[511 - static_cast<int>(x & 511ull)] = 1;
   __syncthreads();
   const bool taken = took[tid] != 0;
   const unsigned ball = __ballot_sync(0xFFFFFFFFu, taken);
