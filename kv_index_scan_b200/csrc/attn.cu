@@ -119,6 +119,8 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnBlocksPerSM) sparse_attn_ke
     const void* __restrict__ q, int q_bf16, RowSrc src, int nsplit, int rows_per_split,
     float scale_log2, float* __restrict__ out, float* __restrict__ lse,
     float* __restrict__ part) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(128) unsigned char attn_smem[];
   const float ninf = -__int_as_float(0x7f800000);
   const int u = blockIdx.x / nsplit;
@@ -353,6 +355,7 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnBlocksPerSM) sparse_attn_ke
 // Merge of the splits of one (r, g): warp h merges head h by log-sum-exp.
 __global__ void attn_combine_kernel(const float* __restrict__ part, int nsplit, int H,
                                     float* __restrict__ out, float* __restrict__ lse) {
+  pdl_wait();
   const int u = blockIdx.x;
   const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (h >= H) return;
@@ -386,9 +389,9 @@ kvs_status launch_h(const void* q, int q_bf16, const RowSrc& src, int RG, int ns
                     float scale_log2, float* out, float* lse, float* part, cudaStream_t s) {
   cudaFuncSetAttribute(sparse_attn_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        kAttnSmem);
-  sparse_attn_kernel<H><<<RG * nsplit, kAttnThreads, kAttnSmem, s>>>(q, q_bf16, src, nsplit, rps,
-                                                                     scale_log2, out, lse, part);
-  if (nsplit > 1) attn_combine_kernel<<<RG, H * 32, 0, s>>>(part, nsplit, H, out, lse);
+  launch_chained(sparse_attn_kernel<H>, dim3(RG * nsplit), dim3(kAttnThreads), kAttnSmem, s, q, q_bf16,
+                 src, nsplit, rps, scale_log2, out, lse, part);
+  if (nsplit > 1) launch_chained(attn_combine_kernel, dim3(RG), dim3(H * 32), 0, s, part, nsplit, H, out, lse);
   return check_launch("sparse_decode_attn");
 }
 

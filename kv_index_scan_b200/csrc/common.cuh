@@ -26,6 +26,33 @@ kvs_status check_launch(const char* what);
     if (!(cond)) return ::kvs::fail(st, __VA_ARGS__); \
   } while (0)
 
+// ----------------------------------------------------------------------------- launch chaining
+// The kernels of a decode step are launched with programmatic stream
+// serialization: a kernel may be launched while its predecessor in the stream
+// still runs (once every block of the predecessor has called pdl_trigger), so
+// that its launch and ramp overlap the predecessor's tail. Every such kernel
+// calls pdl_wait before its first global memory access: it returns once the
+// predecessor has completed and its writes are visible (at once when the
+// kernel was not launched that way).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" :::); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                           Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }

@@ -25,6 +25,8 @@ __global__ void __launch_bounds__(512) plan_bits_kernel(
     const float* __restrict__ kstep, const float* __restrict__ kvar, int B,
     uint8_t* __restrict__ t_out, uint16_t* __restrict__ plane_idx, float* __restrict__ plane_w,
     float* __restrict__ C_out) {
+  pdl_wait();
+  pdl_trigger();
   const int u = blockIdx.x;
   const int tid = threadIdx.x;
   __shared__ float qb[kD], wv[kD];
@@ -126,7 +128,8 @@ __global__ void __launch_bounds__(512) plan_bits_kernel(
 kvs_status plan_bits_launch(const float* q, int H, const float* kmin, const float* kstep,
                             const float* kvar, int RG, int B, uint8_t* t, uint16_t* plane_idx,
                             float* plane_w, float* C, cudaStream_t s) {
-  plan_bits_kernel<<<RG, 512, 0, s>>>(q, H, kmin, kstep, kvar, B, t, plane_idx, plane_w, C);
+  launch_chained(plan_bits_kernel, dim3(RG), dim3(512), 0, s, q, H, kmin, kstep, kvar, B, t, plane_idx,
+                 plane_w, C);
   return check_launch("fathom_plan_bits");
 }
 

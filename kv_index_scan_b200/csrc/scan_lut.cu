@@ -95,6 +95,8 @@ struct LutLaunch {
 // Plans of at most 144 planes: the byte-indexed lookup core (scan_prmt.cuh).
 // Thread t writes the 16 consecutive scores of its half plane word.
 __global__ void __launch_bounds__(kPThreads, 1) fathom_scan_prmt_kernel(ScanParams p) {
+  pdl_wait();
+  pdl_trigger();
   ScanCoreP core(p);
   core.run([&](int u, int c, int nr, const float (&acc)[kPKeys], int t) {
     const int i0 = ScanCoreP::key0(c, t);
@@ -137,7 +139,7 @@ kvs_status fathom_scan_lut_launch(const ScanParams& p, cudaStream_t s) {
     const size_t smem = prmt_smem_bytes(p.B, q.nstage, 0);
     cudaFuncSetAttribute(fathom_scan_prmt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(smem));
-    fathom_scan_prmt_kernel<<<min(chunks, sm_count()), kPThreads, smem, s>>>(q);
+    launch_chained(fathom_scan_prmt_kernel, dim3(min(chunks, sm_count())), dim3(kPThreads), smem, s, q);
     return check_launch("index_scan(fathom, prmt)");
   }
   return dispatch_schedule(p, LutLaunch{p, s});

@@ -755,6 +755,8 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(
     const float* __restrict__ scores, const float* __restrict__ gmax, const int32_t* __restrict__ n,
     int Gheads, int n_max, int k, uint32_t* __restrict__ bitmap, const int32_t* __restrict__ slot_map,
     int32_t* __restrict__ idx, int32_t* __restrict__ slots, int32_t* __restrict__ misses) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ unsigned hist[kTkBins];
   __shared__ TkState st;
   extern __shared__ __align__(16) unsigned char tk_smem[];
@@ -1205,7 +1207,7 @@ kvs_status fathom_scan_topk_launch(ScanParams p, void* ws, const int32_t* slot_m
     if (after_scan) cudaEventRecord(after_scan, s);
     cudaFuncSetAttribute(topk_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kTkSmem));
-    topk_scores_kernel<<<p.RG, kTkThreads, kTkSmem, s>>>(q.scores, q.gmax, p.n, p.Gheads, p.n_max, p.k,
+    launch_chained(topk_scores_kernel, dim3(p.RG), dim3(kTkThreads), kTkSmem, s, q.scores, q.gmax, p.n, p.Gheads, p.n_max, p.k,
                                                          bitmap, slot_map, idx, slots, misses);
     return check_launch("decode_step(top-k over scores)");
   }
