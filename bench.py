@@ -54,9 +54,9 @@ SCAN_KERNEL = "fathom_scan_prmt (scan stage of the step)"
 # the keys processed (the capture and scaling are stated under profiles/);
 # None where no capture of the current kernel exists.
 TRAFFIC: dict = {
-    # R=8 capture of fathom_scan_prmt_kernel: 96.55 MB read + 9.84 MB written
+    # R=8 capture of fathom_scan_prmt_kernel: 96.56 MB read + 9.77 MB written
     # per launch (the rest of its scores leave L2 later), x2 for R=16
-    ("qwen3-8b-128k", 92): 2 * (96_554_240 + 9_842_176),
+    ("qwen3-8b-128k", 92): 2 * (96_558_080 + 9_770_752),
 }
 
 
