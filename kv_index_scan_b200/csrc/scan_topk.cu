@@ -642,7 +642,7 @@ struct TkState {
   uint32_t prefix, mask;
   int krem, done, gt;
   int wcnt[32], ws[32], wt[32];
-  uint32_t wmin[32], wmax[32];
+  uint32_t wmax[32];
   int miss_warp[32];
 };
 
@@ -690,10 +690,11 @@ __device__ uint32_t radix_kth_key(Each&& each, int kk, unsigned* hist, TkState* 
 }
 
 // The same select when every key agrees with `prefix` on the bits above `top`:
-// digits of up to 12 bits from bit `top` down.
+// digits of up to 12 bits from bit `top` down. With first_ready, hist already
+// holds the histogram of the first digit (built while the keys were produced).
 template <typename Each>
-__device__ uint32_t radix_select_from(Each&& each, int top, uint32_t prefix, int kk, unsigned* hist,
-                                      TkState* st, bool* whole, int* gt) {
+__device__ uint32_t radix_select_from(Each&& each, int top, uint32_t prefix, int kk, bool first_ready,
+                                      unsigned* hist, TkState* st, bool* whole, int* gt) {
   const int t = threadIdx.x;
   uint32_t mask = top >= 31 ? 0u : ~((2u << top) - 1u);
   int krem = kk, above = 0;
@@ -702,12 +703,15 @@ __device__ uint32_t radix_select_from(Each&& each, int top, uint32_t prefix, int
     const int shift = top + 1 - width;
     const uint32_t dmask = (1u << width) - 1u;
     const int nb = 1 << width;
-    for (int b = t; b < nb; b += kTkThreads) hist[b] = 0;
-    __syncthreads();
-    each([&](uint32_t key) {
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
-    });
-    __syncthreads();
+    if (!first_ready) {
+      for (int b = t; b < nb; b += kTkThreads) hist[b] = 0;
+      __syncthreads();
+      each([&](uint32_t key) {
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+      });
+      __syncthreads();
+    }
+    first_ready = false;
     find_bin_from_top(hist, nb, krem, st->wsum, st->res, t, kTkThreads, [] { __syncthreads(); });
     const int bin = st->res[0];
     const int ab = st->res[1];
@@ -784,32 +788,38 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(
   uint32_t T = 0u;
   int my_miss = 0;
   if (onchip) {
-    // A. maxima as 16-bit prefixes, with their range; T
-    uint32_t pmin = 0xFFFFu, pmax = 0u;
+    // A. maxima as 16-bit prefixes (the histogram of their bits 15..4 built
+    // as they load) and the largest of them; T
+    for (int b = t; b < kTkBins; b += kTkThreads) hist[b] = 0;
+    __syncthreads();
+    uint32_t pmax = 0u;
 #pragma unroll 8
     for (int g = t; g < m; g += kTkThreads) {
       const uint32_t pfx = ordered_key(__ldg(gm + g)) >> 16;
       gk[g] = static_cast<uint16_t>(pfx);
-      pmin = min(pmin, pfx);
+      atomicAdd(&hist[pfx >> 4], 1u);
       pmax = max(pmax, pfx);
     }
-    pmin = __reduce_min_sync(FULL, pmin);
     pmax = __reduce_max_sync(FULL, pmax);
-    if (lane == 0) {
-      st.wmin[warp] = pmin;
-      st.wmax[warp] = pmax;
-    }
+    if (lane == 0) st.wmax[warp] = pmax;
     __syncthreads();
+    // every key of the row is <= hi (the prefix of its largest maximum, low bits set)
+    const uint32_t hi = (__reduce_max_sync(FULL, st.wmax[lane]) << 16) | 0xFFFFu;
     if (kk <= m) {
-      const uint32_t lo = __reduce_min_sync(FULL, st.wmin[lane]);
-      const uint32_t x = lo ^ __reduce_max_sync(FULL, st.wmax[lane]);
-      const int top = x ? 31 - __clz(x) : 0;
       bool wh;
       int g0;
       T = radix_select_from([&](auto visit) {
             for (int g = t; g < m; g += kTkThreads) visit(static_cast<uint32_t>(gk[g]));
-          }, top, lo & ~((2u << top) - 1u), kk, hist, &st, &wh, &g0) << 16;
+          }, 15, 0u, kk, true, hist, &st, &wh, &g0) << 16;
     }
+    // the candidates lie in [T, hi]: the first digit of their select starts at
+    // the highest bit in which T and hi differ
+    const uint32_t xr = T ^ hi;
+    const int top1 = xr ? 31 - __clz(xr) : 0;
+    const int width1 = min(12, top1 + 1);
+    const int shift1 = top1 + 1 - width1;
+    const uint32_t dmask1 = (1u << width1) - 1u;
+    for (int b = t; b < kTkBins; b += kTkThreads) hist[b] = 0;  // visible after B's barriers
     // B. candidate groups in index order
     const uint32_t Tp = T >> 16;
     int ncg = 0;
@@ -846,10 +856,12 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(
       const int sub = lane >> 2, qtr = lane & 3;
       int wc = 0;
       bool ovf = false;
-      uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
       // four iterations' loads in flight per warp
       constexpr int kU = 4;
       const int niter = (e_end - e_beg + 7) >> 3;
+      // key(v) >= T: for T >= key(+0) one signed compare of v's bits
+      const bool tpos = (T & 0x80000000u) != 0u;
+      const int tint = static_cast<int>(T & 0x7FFFFFFFu);
       for (int it0 = 0; it0 < niter && !ovf; it0 += kU) {
         float4 f[kU];
         int base[kU];
@@ -878,8 +890,10 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(
           uint32_t pass = 0u;
           if (base[a] >= 0) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              if (base[a] + j < nr && ordered_key(v[j]) >= T) pass |= 1u << j;
+            for (int j = 0; j < 4; ++j) {
+              const bool ge = tpos ? __float_as_int(v[j]) >= tint : ordered_key(v[j]) >= T;
+              if (ge && base[a] + j < nr) pass |= 1u << j;
+            }
           }
           const int c = __popc(pass);
           const unsigned b0 = __ballot_sync(FULL, c & 1), b1 = __ballot_sync(FULL, c & 2),
@@ -890,39 +904,28 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(
             break;
           }
           int q = wc + __popc(b0 & lt) + 2 * __popc(b1 & lt) + 4 * __popc(b2 & lt);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if ((pass >> j) & 1u) {
-              const uint32_t key = ordered_key(v[j]);
-              wl[q++] = make_uint2(key, static_cast<uint32_t>(base[a] + j));
-              kmin = min(kmin, key);
-              kmax = max(kmax, key);
-            }
+          while (pass) {
+            const int j = __ffs(pass) - 1;
+            pass &= pass - 1u;
+            const float x = j == 0 ? v[0] : (j == 1 ? v[1] : (j == 2 ? v[2] : v[3]));
+            const uint32_t key = ordered_key(x);
+            wl[q++] = make_uint2(key, static_cast<uint32_t>(base[a] + j));
+            atomicAdd(&hist[(key >> shift1) & dmask1], 1u);
           }
           wc += tot;
         }
       }
-      kmin = __reduce_min_sync(FULL, kmin);
-      kmax = __reduce_max_sync(FULL, kmax);
-      if (lane == 0) {
-        st.wcnt[warp] = ovf ? -1 : wc;
-        st.wmin[warp] = kmin;
-        st.wmax[warp] = kmax;
-      }
+      if (lane == 0) st.wcnt[warp] = ovf ? -1 : wc;
       __syncthreads();
       onchip = !__any_sync(FULL, st.wcnt[lane] < 0);
       if (onchip) {
-        // D. the kk-th largest candidate key
-        const uint32_t lo = __reduce_min_sync(FULL, st.wmin[lane]);
-        const uint32_t hi = __reduce_max_sync(FULL, st.wmax[lane]);
-        const uint32_t x = lo ^ hi;
-        const int top = x ? 31 - __clz(x) : 0;
-        const uint32_t upper = top >= 31 ? 0u : ~((2u << top) - 1u);
+        // D. the kk-th largest candidate key (first digit counted in C)
+        const uint32_t upper = top1 >= 31 ? 0u : ~((2u << top1) - 1u);
         bool whole;
         int gt;
         const uint32_t cut = radix_select_from([&](auto visit) {
               for (int i = lane; i < wc; i += 32) visit(wl[i].x);
-            }, top, lo & upper, kk, hist, &st, &whole, &gt);
+            }, top1, T & upper, kk, true, hist, &st, &whole, &gt);
         // E. ranks in index order: keys above the cut, then the first `need` ties
         const int need = whole ? 0 : kk - gt;
         int ns = 0, nt = 0;

@@ -292,6 +292,49 @@ def test_decode_step_all_tied_long_rows_cut_to_first_indices(kvs):
     assert torch.equal(step.idx.cpu(), torch.arange(k, dtype=torch.int32).expand(R, G, k))
 
 
+@pytest.mark.parametrize("B", [20, 92, 136])
+def test_decode_step_selection_is_exact_topk_of_its_scores(kvs, B):
+    """On ordinary rows (ragged: 100,000 and 131,072 keys) the step's top-k is
+    exactly the k largest of the same scan's scores, ties to the lower index."""
+    R, G, H, n, k = 2, 4, 4, 131072, 2048
+    nl = [100000, n]
+    K, V, _ = synth.fathom_kv(R, G, D, nl, n_max=n, seed=81 + B)
+    q = synth.queries(R, G, H, D, seed=81 + B)
+    ix = kvs.build_fathom_index(K.to(DEV), nl)
+    step = kvs.DecodeStep(ix, nl, n, H, B, k, K.to(DEV), V.to(DEV))
+    step(q.to(DEV))
+    sc = kvs.index_scan_fathom(ix, step.plan, nl, n)
+    torch.cuda.synchronize()
+    order = torch.sort(sc.cpu(), dim=2, descending=True, stable=True).indices[:, :, :k]
+    expect = torch.sort(order, dim=2).values.to(torch.int32)
+    assert torch.equal(step.idx.cpu(), expect)
+
+
+def test_decode_step_high_block_overflows_warp_lists(kvs):
+    """The first 8,192 keys of each row are one key far above the rest: their
+    512 groups are all candidates, and the warps given them collect about
+    1,024 keys each (more than a warp's on-chip list holds) while the number of
+    candidate groups still fits on chip, so the row is selected over global
+    memory. The scores of those keys agree up to the scan's summation order;
+    the selection must be exactly the top-2048 of the same scores (score desc,
+    index asc), all inside the block."""
+    R, G, H, n, k, blk, B = 1, 2, 4, 131072, 2048, 8192, 92
+    K, V, nl = synth.fathom_kv(R, G, D, n, seed=71)
+    q = synth.queries(R, G, H, D, seed=71)
+    s = synth.channel_scales(71, 0, G, D)
+    for g in range(G):
+        K[0, g, :blk] = (3.0 * s[g] * torch.sign(q[0, g].sum(0))).to(torch.bfloat16)
+    ix = kvs.build_fathom_index(K.to(DEV), nl)
+    step = kvs.DecodeStep(ix, nl, n, H, B, k, K.to(DEV), V.to(DEV))
+    step(q.to(DEV))
+    sc = kvs.index_scan_fathom(ix, step.plan, nl, n)
+    torch.cuda.synchronize()
+    order = torch.sort(sc.cpu(), dim=2, descending=True, stable=True).indices[:, :, :k]
+    expect = torch.sort(order, dim=2).values.to(torch.int32)
+    assert torch.equal(step.idx.cpu(), expect)
+    assert int(step.idx.max()) < blk
+
+
 @pytest.mark.parametrize("B", [68, 92])
 def test_host_mapped_index_scan_and_decode(kvs, B):
     """The index planes in mapped pinned host memory, read over the host link
