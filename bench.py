@@ -438,6 +438,87 @@ def run_reference(args, cfg, dist, rank, ws):
             "e2e": {"value": v, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def _time_ms(fn, steps: int, warmup: int) -> float:
+    """Median of per-call CUDA-event times on the current stream."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        fn(0)
+    torch.cuda.synchronize()
+    ts = []
+    for i in range(steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return statistics.median(ts)
+
+
+def run_row(args) -> dict:
+    """Measurements of single rows of the path outside the default decode step
+    (one JSON line each; not the benchmark's headline line):
+      lightning -- the lightning indexer (a2-L) and its block top-k (a3, block
+                   64) at 32 requests x 80000 tokens x 64 index heads;
+      host-scan -- the Fathom scan reading its planes from mapped pinned host
+                   memory (a2-host) at the 1M layer (4 x 8 x 1048576, B = 92),
+                   beside the same scan from HBM and a pinned host-to-device
+                   copy of the same size (the link's copy rate)."""
+    import kv_index_scan_b200 as kvs
+    dev = torch.device("cuda")
+    peak, peak_kind = _peaks()
+    steps, warmup = max(args.steps, 5), max(args.warmup, 3)
+    if args.row == "lightning":
+        R, n, Hi, Dl, block, k = 32, 80000, 64, 128, 64, 2048
+        # two input sets in turn (each 328 MB of index keys, more than L2)
+        sets = [synth.lightning_inputs(R, n, Hi, Dl, seed=3 + j, device=dev) for j in range(2)]
+        nb = (n + block - 1) // block
+        bs = torch.empty(R, nb, dtype=torch.float32, device=dev)
+        scan_ms = _time_ms(lambda i: kvs.index_scan_lightning(*sets[i & 1][:3], sets[i & 1][3],
+                                                               block=block, scores=bs), steps, warmup)
+        idx = torch.empty(R, 1, k, dtype=torch.int32, device=dev)
+        topk_ms = _time_ms(lambda i: kvs.topk_select(bs, sets[0][3], k, block=block, idx=idx),
+                           steps, warmup)
+        kbytes = R * n * Dl
+        flops = 2.0 * R * n * Hi * Dl
+        return {"row": "a2-L lightning indexer + a3 block top-k", "requests": R, "tokens": n,
+                "index_heads": Hi, "block": block, "k": k,
+                "scan_ms": scan_ms, "index_keys_per_s": R * n / (scan_ms / 1e3),
+                "scan_gbs": kbytes / (scan_ms / 1e3) / 1e9, "hbm_peak_gbs": peak, "peak_kind": peak_kind,
+                "scan_frac_hbm": kbytes / (scan_ms / 1e3) / 1e9 / peak,
+                "scan_tflops": flops / (scan_ms / 1e3) / 1e12,
+                "block_topk_ms": topk_ms, "algorithmic_bytes": kbytes, "flops": flops}
+    if args.row == "host-scan":
+        R, G, n, B = 4, 8, 1048576, 92
+        K, _, nl = synth.fathom_kv(R, G, 128, n, seed=2, device=dev, with_v=False)
+        q = synth.queries(R, G, 4, 128, seed=2, device=dev)
+        ix = kvs.build_fathom_index(K, nl)
+        del K
+        plan = kvs.fathom_plan_bits(q, ix, B)
+        scores = torch.empty(R, G, n, dtype=torch.float32, device=dev)
+        hbm_ms = _time_ms(lambda i: kvs.index_scan_fathom(ix, plan, nl, n, scores=scores), steps, warmup)
+        ref = scores.clone()
+        hix = kvs.MappedHostIndex(ix)
+        host_ms = _time_ms(lambda i: kvs.index_scan_fathom(hix, plan, nl, n, scores=scores),
+                           min(steps, 10), 2)
+        host_vs_hbm = float((ref - scores).abs().max())
+        plane_bytes = R * G * n * B / 8
+        # the link's copy rate for the same byte count, from pinned host memory
+        host_buf = torch.empty(int(plane_bytes), dtype=torch.uint8).pin_memory()
+        dev_buf = torch.empty(int(plane_bytes), dtype=torch.uint8, device=dev)
+        copy_ms = _time_ms(lambda i: dev_buf.copy_(host_buf, non_blocking=True), 5, 2)
+        return {"row": "a2-host Fathom scan over mapped pinned host memory", "requests": R,
+                "kv_heads": G, "context": n, "bits_per_key": B, "plane_bytes": plane_bytes,
+                "hbm_scan_ms": hbm_ms, "hbm_keys_per_s": R * G * n / (hbm_ms / 1e3),
+                "hbm_scan_gbs": plane_bytes / (hbm_ms / 1e3) / 1e9, "hbm_frac": plane_bytes / (hbm_ms / 1e3) / 1e9 / peak,
+                "host_scan_ms": host_ms, "host_keys_per_s": R * G * n / (host_ms / 1e3),
+                "host_link_gbs": plane_bytes / (host_ms / 1e3) / 1e9,
+                "pinned_copy_gbs": plane_bytes / (copy_ms / 1e3) / 1e9,
+                "host_link_frac_of_copy": copy_ms / host_ms,
+                "max_abs_diff_vs_hbm_scan": host_vs_hbm}
+    raise ValueError(args.row)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -453,7 +534,12 @@ def main():
     ap.add_argument("--only-step", action="store_true",
                     help="time the decode steps only (no scan-alone, end-to-end or CPU legs); "
                          "prints the step and stage times, for profiling runs")
+    ap.add_argument("--row", default=None, choices=["lightning", "host-scan"],
+                    help="measure one row of the path outside the decode step (one JSON line)")
     args = ap.parse_args()
+    if args.row is not None:
+        print(json.dumps(run_row(args)), flush=True)
+        return
     cfg = dict(WORKLOADS[args.workload])
     if args.B is not None:
         cfg["B"] = args.B

@@ -12,17 +12,20 @@
 // the 5th-generation tensor cores:
 //  * a producer warp streams 128-token e4m3 tiles (16 KB, one 1-D TMA bulk
 //    copy each) into a shared-memory ring;
-//  * four converter warps turn each tile into f16 (exact for e4m3) in the
+//  * sixteen converter warps turn each tile into f16 (exact for e4m3) in the
 //    canonical 128-byte-swizzled K-major layout of the MMA's A operand; the
 //    queries become the B operand once per request, in f16 after scaling by a
 //    power of two (exact) that brings max|q| to [2^13, 2^14);
 //  * one elected thread issues tcgen05.mma kind::f16 (M = 128 tokens,
-//    N = Hi heads, K = 16 per instruction, 8 instructions) into one of two
+//    N = Hi heads, K = 16 per instruction, 8 instructions) into one of three
 //    f32 accumulators in tensor memory, and commits to mbarriers;
 //  * the converter warps then read the accumulators back (tcgen05.ld: one
-//    token row per thread), apply ReLU, the head weights (with the scale
-//    undone) and the head sum, and reduce 32/64/128-token blocks with warp
-//    shuffles.
+//    token row per thread; warp w reads the TMEM lanes of tokens
+//    32 (w mod 4) .. + 31 and the 16-head column chunks c = w / 4, w / 4 + 4),
+//    apply ReLU and the head weights (with the scale undone); the four partial
+//    head sums of a token meet in shared memory, and warps 0-3 reduce
+//    32/64/128-token blocks with warp shuffles. (Four warps, one per
+//    scheduler, left the conversion and read-back latency-bound.)
 // Every wait is bounded; a wait that runs out sets KVS_ETIMEOUT in the status
 // word and the block winds down without leaving copies in flight or TMEM
 // allocated.
@@ -37,21 +40,29 @@ namespace {
 constexpr int kTileTok = 128;                 // tokens per tile (MMA M)
 constexpr int kRawBytes = kTileTok * 128;      // e4m3 tile: 128 tokens x 128 channels
 constexpr int kATileBytes = kTileTok * 256;    // f16 tile, two 128-byte-wide K blocks
-constexpr int kNRaw = 4;                       // raw tile ring depth
-constexpr int kLThreads = 192;                 // warps 0-3 convert + epilogue, 4 load, 5 MMA
+constexpr int kNRaw = 3;                       // raw tile ring depth
+constexpr int kNAcc = 3;                       // A tiles and accumulators in flight
+constexpr int kLConvWarps = 16;                // warps 0-15 convert + epilogue
+constexpr int kLConv = 32 * kLConvWarps;
+constexpr int kLoadWarp = kLConvWarps, kMmaWarp = kLConvWarps + 1;
+constexpr int kLThreads = kLConv + 64;
 constexpr long long kLWaitCycles = 2000000000ll;
 
 struct LSmem {
-  alignas(1024) unsigned char a[2][kATileBytes];    // converted A tiles (SW128 K-major)
+  alignas(1024) unsigned char a[kNAcc][kATileBytes];  // converted A tiles (SW128 K-major)
   alignas(1024) unsigned char bq[2][128 * 256];     // query B operand per request parity
   alignas(1024) unsigned char raw[kNRaw][kRawBytes];
-  float w[2][128];                                  // weights (scale undone) per request parity
-  float blockpart[2][4];                            // per-warp block maxima
-  float qmax[4];
-  uint64_t raw_full[kNRaw], raw_empty[kNRaw], a_full[2], a_empty[2], acc_full[2], acc_empty[2];
+  float w[4][128];                                  // weights (scale undone), request sequence mod 4
+  float spart[kNAcc][4][kTileTok];                  // partial head sums per column group
+  float blockpart[kNAcc][4];                        // per-warp block maxima
+  float qmax[kLConvWarps];
+  uint64_t raw_full[kNRaw], raw_empty[kNRaw], a_full[kNAcc], a_empty[kNAcc], acc_full[kNAcc],
+      acc_empty[kNAcc];
   uint32_t tmem_base;
   int abort_flag;
 };
+
+static_assert(sizeof(LSmem) + 1024 <= 227 * 1024, "lightning shared memory over the per-block limit");
 
 __device__ __forceinline__ uint32_t saddr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -90,8 +101,11 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       "l"(src), "r"(bytes), "r"(saddr(bar))
       : "memory");
 }
-__device__ __forceinline__ void group_sync() {  // the four converter / epilogue warps
-  asm volatile("bar.sync 2, 128;\n" ::: "memory");
+__device__ __forceinline__ void group_sync() {  // the converter / epilogue warps
+  asm volatile("bar.sync 2, %0;\n" ::"n"(kLConv) : "memory");
+}
+__device__ __forceinline__ void tile_sync() {  // warps 0-3: one tile's 128 tokens
+  asm volatile("bar.sync 3, 128;\n" ::: "memory");
 }
 
 // Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzle
@@ -165,23 +179,24 @@ __global__ void __launch_bounds__(kLThreads, 1) lightning_scan_kernel(LParams p)
   const int beg = static_cast<int>(static_cast<long long>(blockIdx.x) * T / gridDim.x);
   const int end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * T / gridDim.x);
   const int Hi = p.Hi;
-  const uint32_t tmem_cols = Hi <= 64 ? 128u : 256u;  // two accumulators of Hi columns
+  // kNAcc accumulators of Hi columns (a power of two >= 32 columns)
+  const uint32_t tmem_cols = Hi <= 32 ? 128u : (Hi <= 64 ? 256u : 512u);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNRaw; ++i) {
       bar_init(&sm.raw_full[i], 1);
-      bar_init(&sm.raw_empty[i], 4);
+      bar_init(&sm.raw_empty[i], kLConvWarps);
     }
-    for (int i = 0; i < 2; ++i) {
-      bar_init(&sm.a_full[i], 4);
+    for (int i = 0; i < kNAcc; ++i) {
+      bar_init(&sm.a_full[i], kLConvWarps);
       bar_init(&sm.a_empty[i], 1);
       bar_init(&sm.acc_full[i], 1);
-      bar_init(&sm.acc_empty[i], 4);
+      bar_init(&sm.acc_empty[i], kLConvWarps);
     }
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
                      saddr(&sm.tmem_base)),
                  "r"(tmem_cols)
@@ -199,7 +214,7 @@ __global__ void __launch_bounds__(kLThreads, 1) lightning_scan_kernel(LParams p)
   };
   auto aborted = [&] { return *reinterpret_cast<volatile int*>(&sm.abort_flag) != 0; };
 
-  if (warp == 4) {
+  if (warp == kLoadWarp) {
     // ---------------- producer: raw e4m3 tiles ----------------
     if (lane == 0) {
       int issued = 0;
@@ -224,7 +239,7 @@ __global__ void __launch_bounds__(kLThreads, 1) lightning_scan_kernel(LParams p)
       for (int i = max(0, issued - kNRaw); i < issued; ++i)
         bar_wait(&sm.raw_full[i % kNRaw], (i / kNRaw) & 1);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t idesc = (1u << 4) | (static_cast<uint32_t>(Hi >> 3) << 17) | (8u << 24);
@@ -236,12 +251,12 @@ __global__ void __launch_bounds__(kLThreads, 1) lightning_scan_kernel(LParams p)
           ++req_seq;
           prev_r = r;
         }
-        const int x = i & 1;
-        if (!bar_wait(&sm.a_full[x], (i >> 1) & 1)) {
+        const int x = i % kNAcc;
+        if (!bar_wait(&sm.a_full[x], (i / kNAcc) & 1)) {
           fail();
           break;
         }
-        if (i >= 2 && !bar_wait(&sm.acc_empty[x], ((i >> 1) - 1) & 1)) {
+        if (i >= kNAcc && !bar_wait(&sm.acc_empty[x], ((i / kNAcc) - 1) & 1)) {
           fail();
           break;
         }
@@ -260,7 +275,7 @@ __global__ void __launch_bounds__(kLThreads, 1) lightning_scan_kernel(LParams p)
       }
     }
   } else {
-    // ---------------- converters + epilogue (warps 0-3) ----------------
+    // ---------------- converters + epilogue (warps 0-15) ----------------
     const int t = threadIdx.x;
     int req_seq = -1, prev_r = -1;
     bool dead = false;
@@ -268,20 +283,21 @@ __global__ void __launch_bounds__(kLThreads, 1) lightning_scan_kernel(LParams p)
       const int tile = beg + i;
       const int r = tile / p.tiles_per_req, t0 = (tile % p.tiles_per_req) * kTileTok;
       const int nr = p.n[r];
-      const int x = i & 1;
-      // request parity of tile i: recomputed from the tiles' request sequence
-      int seq = 0, rr = beg / p.tiles_per_req;
-      seq = r - rr;  // consecutive requests in a contiguous tile range
-      const float* wv = sm.w[seq & 1];
+      const int x = i % kNAcc;
+      // request sequence of tile i (consecutive requests in a contiguous tile range)
+      const int seq = r - beg / p.tiles_per_req;
+      const float* wv = sm.w[seq & 3];
+      const int quarter = warp & 3, cgrp = warp >> 2;
+      const int tin = quarter * 32 + lane;  // this thread's token (TMEM lane) in the tile
       float S = 0.f;
-      if (!dead && bar_wait(&sm.acc_full[x], (i >> 1) & 1)) {
+      if (!dead && bar_wait(&sm.acc_full[x], (i / kNAcc) & 1)) {
         tc_fence_after();
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(x * Hi);
-        for (int c0 = 0; c0 < Hi; c0 += 16) {
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(x * Hi);
+        for (int c = cgrp; c < Hi / 16; c += 4) {
           float v[16];
-          tmem_ld16(taddr + static_cast<uint32_t>(c0), v);
+          tmem_ld16(taddr + static_cast<uint32_t>(16 * c), v);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) S = fmaf(wv[c0 + e], fmaxf(v[e], 0.f), S);
+          for (int e = 0; e < 16; ++e) S = fmaf(wv[16 * c + e], fmaxf(v[e], 0.f), S);
         }
         tc_fence_before();
       } else if (!dead) {
@@ -290,7 +306,11 @@ __global__ void __launch_bounds__(kLThreads, 1) lightning_scan_kernel(LParams p)
       }
       __syncwarp();
       if (lane == 0 && !dead) bar_arrive(&sm.acc_empty[x]);
-      const int tok = t0 + t;
+      sm.spart[x][cgrp][tin] = S;
+      group_sync();
+      if (cgrp != 0) return;
+      S = (sm.spart[x][0][tin] + sm.spart[x][1][tin]) + (sm.spart[x][2][tin] + sm.spart[x][3][tin]);
+      const int tok = t0 + tin;
       const float ninf = -__int_as_float(0x7f800000);
       float v = tok < nr ? S : ninf;
       float* out = p.out + static_cast<size_t>(r) * p.nb_max;
@@ -306,7 +326,7 @@ __global__ void __launch_bounds__(kLThreads, 1) lightning_scan_kernel(LParams p)
       }
       // 64- or 128-token blocks span 2 or 4 warps
       if (lane == 0) sm.blockpart[x][warp] = v;
-      group_sync();
+      tile_sync();
       if (lane == 0) {
         const int per = p.block / 32;
         if (warp % per == 0) {
@@ -315,29 +335,37 @@ __global__ void __launch_bounds__(kLThreads, 1) lightning_scan_kernel(LParams p)
           if (tok < p.n_max) out[tok / p.block] = m;
         }
       }
-      group_sync();
+      tile_sync();
     };
     for (int i = 0; i < end - beg; ++i) {
       const int tile = beg + i;
       const int r = tile / p.tiles_per_req;
-      const int x = i & 1;
+      const int x = i % kNAcc;
       const int st = i % kNRaw;
-      if (i >= 2 && !dead && !bar_wait(&sm.a_empty[x], ((i >> 1) - 1) & 1)) {
+      if (i >= kNAcc && !dead && !bar_wait(&sm.a_empty[x], ((i / kNAcc) - 1) & 1)) {
         fail();
         dead = true;
       }
       if (r != prev_r) {
         ++req_seq;
         prev_r = r;
+        // the MMAs of the two previous tiles may still read the query buffer
+        // of this parity: wait for them (a request has one tile at least)
+        for (int j = max(0, i - 2); j < i && !dead; ++j)
+          if (!bar_wait(&sm.a_empty[j % kNAcc], (j / kNAcc) & 1)) {
+            fail();
+            dead = true;
+          }
         // the request's queries as the B operand, scaled by 2^e into f16
         const int par = req_seq & 1;
         const uint16_t* q = p.qidx + static_cast<size_t>(r) * Hi * 128;
         float mx = 0.f;
-        for (int e = t; e < Hi * 128; e += 128) mx = fmaxf(mx, fabsf(bf16_bits_to_float(q[e])));
+        for (int e = t; e < Hi * 128; e += kLConv) mx = fmaxf(mx, fabsf(bf16_bits_to_float(q[e])));
         for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, d));
         if (lane == 0) sm.qmax[warp] = mx;
         group_sync();
-        mx = fmaxf(fmaxf(sm.qmax[0], sm.qmax[1]), fmaxf(sm.qmax[2], sm.qmax[3]));
+        mx = 0.f;
+        for (int e = 0; e < kLConvWarps; ++e) mx = fmaxf(mx, sm.qmax[e]);
         int ex = 0;
         if (mx > 0.f) {
           int e2;
@@ -345,7 +373,7 @@ __global__ void __launch_bounds__(kLThreads, 1) lightning_scan_kernel(LParams p)
           ex = 14 - e2;     // scaled max in [2^13, 2^14)
         }
         const float sc = ldexpf(1.f, ex), inv = ldexpf(1.f, -ex);
-        for (int c = t; c < Hi * 16; c += 128) {  // 16-byte output chunks: row h, chunk cc
+        for (int c = t; c < Hi * 16; c += kLConv) {  // 16-byte output chunks: row h, chunk cc
           const int h = c >> 4, cc = c & 15;
           const uint16_t* src = q + h * 128 + cc * 8;
           uint32_t packed[4];
@@ -360,7 +388,7 @@ __global__ void __launch_bounds__(kLThreads, 1) lightning_scan_kernel(LParams p)
           *reinterpret_cast<uint4*>(sm.bq[par] + kb * (Hi * 128) + sw128_off(h, j)) =
               make_uint4(packed[0], packed[1], packed[2], packed[3]);
         }
-        for (int h = t; h < Hi; h += 128) sm.w[par][h] = p.w[static_cast<size_t>(r) * Hi + h] * inv;
+        for (int h = t; h < Hi; h += kLConv) sm.w[req_seq & 3][h] = p.w[static_cast<size_t>(r) * Hi + h] * inv;
       }
       // convert the raw tile into the swizzled f16 A tile
       if (!dead && !bar_wait(&sm.raw_full[st], (i / kNRaw) & 1)) {
@@ -368,7 +396,7 @@ __global__ void __launch_bounds__(kLThreads, 1) lightning_scan_kernel(LParams p)
         dead = true;
       }
       if (!dead) {
-        for (int c = t; c < kTileTok * 8; c += 128) {  // 16-byte raw chunk: row, part
+        for (int c = t; c < kTileTok * 8; c += kLConv) {  // 16-byte raw chunk: row, part
           const int row = c >> 3, part = c & 7;
           const uint4 raw = *reinterpret_cast<const uint4*>(sm.raw[st] + row * 128 + part * 16);
           const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -396,14 +424,16 @@ __global__ void __launch_bounds__(kLThreads, 1) lightning_scan_kernel(LParams p)
           bar_arrive(&sm.a_full[x]);
         }
       }
-      if (i >= 1) epilogue(i - 1);
+      // the read-back runs two tiles behind the conversion, so that a tile's
+      // MMAs have a whole conversion period to complete
+      if (i >= 2) epilogue(i - 2);
     }
-    if (end - beg >= 1) epilogue(end - beg - 1);
+    for (int j = max(0, end - beg - 2); j < end - beg; ++j) epilogue(j);
   }
   // wind down: TMEM is released by the warp that allocated it
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(tmem_cols)
                  : "memory");
