@@ -39,6 +39,13 @@
  *     synchronises; it only enqueues kernels on `stream` (a cudaStream_t,
  *     NULL = the legacy default stream). Calls are therefore safe to capture
  *     in a CUDA graph, like the caller-owned top-k buffer of [MINIMAX].
+ *   - Stream order holds as usual: a call's kernels start their memory
+ *     accesses only after the work enqueued before them on `stream` has
+ *     completed. The kernels of one decode_step (and the Fathom scan, the
+ *     top-k over scores and the attention) are launched with programmatic
+ *     stream serialization: the next kernel may be scheduled while its
+ *     predecessor finishes, but waits for it (griddepcontrol.wait) before
+ *     its first global access.
  *   - Scratch memory comes from the caller's workspace `ws` of `ws_bytes`
  *     bytes (16-byte aligned); its required size is returned by the matching
  *     kvs_*_workspace_size() query. ws_bytes too small -> KVS_EWORKSPACE.
