@@ -275,15 +275,20 @@ KVS_API size_t kvs_attn_workspace_size(int32_t R, int32_t G, int32_t H, int32_t 
  *
  * Its scratch (the split-K partial results) is one fixed 4 MiB device array
  * inside this library, which every GPU that loads the library holds until the
- * process exits. The need is kvs_attn_workspace_size() and stays below
- * 8 * (SM count) * H * 528 bytes; on a 148-SM B200 every size with H <= 4
- * fits. Sizes that need more are rejected with KVS_EINVAL and a message. The call allocates nothing and calls no
- * allocator. The first call on each device looks up that device's address of
- * the array (with the device current); make that first call before any
- * stream capture. Every call shares the array: nothing in it has to start at
- * zero (each split writes its whole partial before the merge reads it), but
- * calls that overlap on the same GPU (other streams, other host threads)
- * race on it and must be serialised by the caller. */
+ * process exits. Each call cuts the k rows into the cheapest number of splits
+ * whose partial results fit in that array (R*G*splits*H*132 floats; a single
+ * split per (r, g) needs none), so every size is accepted: sizes for which
+ * sparse_decode_attn would use more splits than fit run with fewer, at some
+ * cost in speed. KVS_EINVAL with a message is returned only for argument
+ * errors (and, defensively, if a split ever needed more than the array). The
+ * call allocates nothing and calls no allocator. The first call on each
+ * device looks up that device's address of the array (with the device
+ * current) and caches it for the life of the process (the cache does not
+ * survive cudaDeviceReset); make that first call before any stream capture.
+ * Every call shares the array: nothing in it has to start at zero (each split
+ * writes its whole partial before the merge reads it), but calls that overlap
+ * on the same GPU (other streams, other host threads) race on it and must be
+ * serialised by the caller. */
 KVS_API kvs_status sparse_decode_attn_noalloc(const void* q, int32_t q_dtype, const uint16_t* K,
                                               const uint16_t* V, const int32_t* k_eff, int32_t R,
                                               int32_t G, int32_t H, int32_t D, int32_t k,
@@ -293,9 +298,15 @@ KVS_API kvs_status sparse_decode_attn_noalloc(const void* q, int32_t q_dtype, co
 /* ---------------------------------------------------------------------------
  * a6: one fused decode step for all (r, g), on one stream.
  *
- * idx_in == NULL: a1 (plan into `plan`), a2 with the top-k candidates kept
- *   per chunk on chip (no score array), a3 merge into idx, then a5 reading K/V
- *   straight through slot_map (a4 without staging), misses counted.
+ * idx_in == NULL: a1 (plan into `plan`), then a2 and a3. For plans of at
+ *   most 144 planes the scan writes every score and the maximum of every
+ *   16-key group into the workspace, and a per-row top-k kernel bounds the
+ *   k-th score by the k-th largest group maximum, reads back only the groups
+ *   that can hold a selected key and selects exactly (ties to the lower
+ *   index), writing idx, the slots and the miss counts. For longer plans the
+ *   scan keeps top-k candidates per chunk on chip and a per-row merge selects
+ *   from them. Then a5 reads K/V straight through slot_map (a4 without
+ *   staging), misses counted.
  * idx_in != NULL: the selection is reused and a1..a3 are skipped -- the layer
  *   sharing of [MINIMAX], where a group's first layer selects and the others
  *   reuse it. idx_shared = 1 means idx_in is [R][k], one row per request

@@ -333,12 +333,31 @@ def sparse_decode_attn(q, K, V, k_eff=None, scale: float | None = None, want_lse
     return out, lse
 
 
+def _require(cond: bool, what: str):
+    if not cond:
+        raise ValueError(what)
+
+
 def sparse_decode_attn_noalloc(q, K, V, out, lse=None, k_eff=None, scale: float | None = None,
                                stream=None, dev_status=None):
     """a5 without a workspace, into caller-provided out (and lse): the library
-    keeps the split-K scratch in a fixed device array (see include/kvscan.h)."""
+    keeps the split-K scratch in a fixed device array (see include/kvscan.h).
+    out must be f32 [R][G][H][D] and lse f32 [R][G][H], contiguous, on q's
+    device; k_eff (nullable) int32 [R][G]."""
     R, G, H, D = q.shape
     k = K.shape[2]
+    for name, t, shape, dt in (("out", out, (R, G, H, D), torch.float32),
+                               ("lse", lse, (R, G, H), torch.float32),
+                               ("k_eff", k_eff, (R, G), torch.int32)):
+        if t is None:
+            _require(name != "out", "out is required")
+            continue
+        _require(t.dtype == dt, f"{name} must be {dt}, got {t.dtype}")
+        _require(tuple(t.shape) == shape, f"{name} must have shape {shape}, got {tuple(t.shape)}")
+        _require(t.is_contiguous(), f"{name} must be contiguous")
+        _require(t.device == q.device, f"{name} must be on {q.device}")
+    _require(tuple(K.shape) == (R, G, k, D) and tuple(V.shape) == (R, G, k, D),
+             "K and V must be [R][G][k][D]")
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     qd = KVS_BF16 if q.dtype == torch.bfloat16 else KVS_F32
     st = _lib.sparse_decode_attn_noalloc(_ptr(_u16(q)), qd, _ptr(_u16(K)), _ptr(_u16(V)), _ptr(k_eff),

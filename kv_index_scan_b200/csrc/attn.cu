@@ -399,8 +399,11 @@ kvs_status launch_h(const void* q, int q_bf16, const RowSrc& src, int RG, int ns
 
 // Split of the k rows across blocks: the split count that minimises (waves of
 // blocks) x (64-row units per block + one unit of per-block overhead), ties to
-// fewer splits.
-void attn_split(int RG, int k, int& nsplit, int& rows_per_split) {
+// fewer splits. With max_part_bytes > 0 only the splits whose partial results
+// (RG * nsplit * H * (128 + 4) floats) fit in that many bytes are considered;
+// one split needs none, so there is always one.
+static void attn_split_impl(int RG, int H, int k, size_t max_part_bytes, int& nsplit,
+                            int& rows_per_split) {
   const int units = max(1, (k + kSplitUnit - 1) / kSplitUnit);
   const long long slots = static_cast<long long>(kAttnBlocksPerSM) * sm_count();
   int best = 1;
@@ -408,6 +411,9 @@ void attn_split(int RG, int k, int& nsplit, int& rows_per_split) {
   for (int ns = 1; ns <= min(units, 64); ++ns) {
     const int per = (units + ns - 1) / ns;
     const int used = (units + per - 1) / per;
+    if (max_part_bytes > 0 && used > 1 &&
+        static_cast<size_t>(RG) * used * H * (kD + 4) * sizeof(float) > max_part_bytes)
+      continue;
     const long long waves = (static_cast<long long>(RG) * used + slots - 1) / slots;
     const long long cost = waves * (per + 1);
     if (best_cost < 0 || cost < best_cost) {
@@ -420,6 +426,10 @@ void attn_split(int RG, int k, int& nsplit, int& rows_per_split) {
   nsplit = (units + per - 1) / per;
 }
 
+void attn_split(int RG, int k, int& nsplit, int& rows_per_split) {
+  attn_split_impl(RG, 1, k, 0, nsplit, rows_per_split);
+}
+
 size_t attn_ws_bytes(int RG, int H, int k) {
   int nsplit, rps;
   attn_split(RG, k, nsplit, rps);
@@ -427,11 +437,9 @@ size_t attn_ws_bytes(int RG, int H, int k) {
   return static_cast<size_t>(RG) * nsplit * H * (kD + 4) * sizeof(float);
 }
 
-kvs_status attn_launch(const void* q, int q_bf16, const RowSrc& src, int RG, int H, float scale,
-                       float* out, float* lse, void* ws, cudaStream_t s) {
-  int nsplit, rps;
-  attn_split(RG, src.k, nsplit, rps);
-  float* part = static_cast<float*>(ws);
+static kvs_status attn_launch_split(const void* q, int q_bf16, const RowSrc& src, int RG, int H,
+                                    float scale, float* out, float* lse, float* part, int nsplit,
+                                    int rps, cudaStream_t s) {
   const float sl2 = scale * 1.4426950408889634f;
   switch (H) {
     case 1: return launch_h<1>(q, q_bf16, src, RG, nsplit, rps, sl2, out, lse, part, s);
@@ -446,6 +454,26 @@ kvs_status attn_launch(const void* q, int q_bf16, const RowSrc& src, int RG, int
   }
 }
 
+kvs_status attn_launch(const void* q, int q_bf16, const RowSrc& src, int RG, int H, float scale,
+                       float* out, float* lse, void* ws, cudaStream_t s) {
+  int nsplit, rps;
+  attn_split(RG, src.k, nsplit, rps);
+  return attn_launch_split(q, q_bf16, src, RG, H, scale, out, lse, static_cast<float*>(ws), nsplit,
+                           rps, s);
+}
+
+// The attention with a split whose partial results fit in part_bytes (the
+// cheapest such split; one split writes none). *need receives the bytes used.
+kvs_status attn_launch_fit(const void* q, int q_bf16, const RowSrc& src, int RG, int H,
+                           float scale, float* out, float* lse, float* part, size_t part_bytes,
+                           size_t* need, cudaStream_t s) {
+  int nsplit, rps;
+  attn_split_impl(RG, H, src.k, part_bytes, nsplit, rps);
+  *need = nsplit > 1 ? static_cast<size_t>(RG) * nsplit * H * (kD + 4) * sizeof(float) : 0;
+  if (*need > part_bytes) return fail(KVS_EINVAL, "attention split needs %zu bytes, %zu available", *need, part_bytes);
+  return attn_launch_split(q, q_bf16, src, RG, H, scale, out, lse, part, nsplit, rps, s);
+}
+
 }  // namespace kvs
 
 // ----------------------------------------------------------------------------
@@ -457,13 +485,11 @@ kvs_status attn_launch(const void* q, int q_bf16, const RowSrc& src, int RG, int
 
 namespace {
 
-// 4 MiB of partial results: R*G*nsplit*H*(128+4) floats, none when one split
-// per (r, g) suffices. On a 148-SM B200 at k = 2048 and H = 4 the need is
-// 0.5 MiB up to R*G = 296 (the batches of a decode step) and passes 4 MiB from
-// about R*G = 512 up to 2047, where the rows are cut into several splits;
-// from R*G = 2048 one split suffices and the need is zero. Larger needs are
-// rejected. Every GPU that loads this library holds the array until the
-// process exits.
+// 4 MiB of partial results: R*G*nsplit*H*(128+4) floats. Each call takes the
+// cheapest split of the k rows whose partial results fit here; one split per
+// (r, g) writes none, so every size runs (sizes whose workspace split would
+// need more than 4 MiB run with fewer splits). Every GPU that loads this
+// library holds the array until the process exits.
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 static __device__ __align__(256) float g_attn_scratch[kNoAllocScratchBytes / sizeof(float)];
 
@@ -472,7 +498,9 @@ float* g_scratch_dev[64] = {nullptr};
 
 // Device address of g_attn_scratch on the current device. The name of the
 // array in host code is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// once per device (with that device current) and cached for the life of the
+// process; the cache does not survive cudaDeviceReset (after a reset, reload
+// the library before calling again).
 kvs_status noalloc_scratch(float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -508,11 +536,6 @@ extern "C" kvs_status sparse_decode_attn_noalloc(const void* q, int32_t q_dtype,
   KVS_REQUIRE(D == kD, KVS_EUNSUPPORTED, "sparse_decode_attn_noalloc: D=%d (only 128 is built)", D);
   KVS_REQUIRE(aligned16(K) && aligned16(V) && aligned16(out), KVS_EINVAL,
               "sparse_decode_attn_noalloc: K, V and out must be 16-byte aligned");
-  const size_t need = attn_ws_bytes(R * G, H, k);
-  KVS_REQUIRE(need <= kNoAllocScratchBytes, KVS_EINVAL,
-              "sparse_decode_attn_noalloc: R=%d G=%d H=%d k=%d needs %zu bytes of scratch, more "
-              "than the fixed %zu-byte array; use sparse_decode_attn with a workspace",
-              R, G, H, k, need, kNoAllocScratchBytes);
   float* scratch = nullptr;
   kvs_status st = noalloc_scratch(&scratch);
   if (st != KVS_OK) return st;
@@ -523,7 +546,13 @@ extern "C" kvs_status sparse_decode_attn_noalloc(const void* q, int32_t q_dtype,
   src.k_eff = k_eff;
   src.G = G;
   src.k = k;
-  st = attn_launch(q, q_dtype == KVS_BF16, src, R * G, H, scale, out, lse, scratch,
-                   static_cast<cudaStream_t>(stream));
+  size_t need = 0;
+  st = attn_launch_fit(q, q_dtype == KVS_BF16, src, R * G, H, scale, out, lse, scratch,
+                       kNoAllocScratchBytes, &need, static_cast<cudaStream_t>(stream));
+  if (st == KVS_EINVAL)
+    return fail(KVS_EINVAL,
+                "sparse_decode_attn_noalloc: R=%d G=%d H=%d k=%d needs %zu bytes of scratch, more "
+                "than the fixed %zu-byte array",
+                R, G, H, k, need, kNoAllocScratchBytes);
   return st == KVS_OK ? ok() : st;
 }

@@ -62,6 +62,9 @@ void attn_split(int RG, int k, int& nsplit, int& rows_per_split);
 size_t attn_ws_bytes(int RG, int H, int k);
 kvs_status attn_launch(const void* q, int q_bf16, const RowSrc& src, int RG, int H, float scale,
                        float* out, float* lse, void* ws, cudaStream_t s);
+kvs_status attn_launch_fit(const void* q, int q_bf16, const RowSrc& src, int RG, int H,
+                           float scale, float* out, float* lse, float* part, size_t part_bytes,
+                           size_t* need, cudaStream_t s);
 size_t decode_ws_bytes(int R, int G, int H, int n_max, int k, int B);
 kvs_status decode_step_run(const kvs_decode_args* a, void* ws, int32_t* dev_status,
                            cudaStream_t s,

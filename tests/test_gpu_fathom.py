@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import synth
-from tests._parity import ATTN_TOL, check_selection, fathom_score_tol
+from tests._parity import ATTN_TOL, check_row_over_selection, check_selection, fathom_score_tol
 
 pytestmark = pytest.mark.gpu
 D = 128
@@ -207,6 +207,7 @@ def _decode_case(kvs, R, G, H, nl, n_max, B, k, S, seed, rows=None):
     hotK, hotV = synth.hot_rows(K, hot_tok), synth.hot_rows(V, hot_tok)
     ref = oracle.decode_batch(q, planes, kmin, kstep, kvar, nl, B, k, slot_map, hotK, hotV, K, V,
                               scale, rows=rows, want_scores=True)
+    ref.update(q=q, K=K, V=V, slot_map=slot_map, hotK=hotK, hotV=hotV, scale=scale)
     ix = kvs.build_fathom_index(K.to(DEV), nl, W)
     step = kvs.DecodeStep(ix, nl, n_max, H, B, k, K.to(DEV), V.to(DEV),
                           torch.from_numpy(slot_map).to(DEV), hotK.to(DEV), hotV.to(DEV))
@@ -215,22 +216,34 @@ def _decode_case(kvs, R, G, H, nl, n_max, B, k, S, seed, rows=None):
     return ref, step
 
 
-def _check_decode(ref, step, R, G, nl, k, rows=None):
+def _check_decode(ref, step, R, G, nl, k, rows=None, max_diff_frac=1e-3):
+    """Every listed row: allocation bit-exact, selection equal to the oracle's
+    or differing only inside the tie band, and slots, misses and attention
+    against the oracle's gather and attention over the GPU's own selection
+    (rows whose selection differs are checked too). Returns the number of
+    differing selected entries, which is printed and bounded."""
     t, idx, slots, misses = _np(step.plan.t), _np(step.idx), _np(step.slots), _np(step.misses)
     out, lse = _np(step.out), _np(step.lse)
     rows = range(R * G) if rows is None else rows
-    diffs = 0
+    diffs = diff_rows = entries = 0
     for u in rows:
         r, g = divmod(u, G)
         ke = min(k, nl[r])
         assert np.array_equal(t[r, g], ref["t"][r, g])
         d = check_selection(idx[r, g], ref["idx"][r, g], ref["scores"][r, g, : nl[r]], ke)
         diffs += d
+        diff_rows += d > 0
+        entries += ke
         if d == 0:
             assert np.array_equal(slots[r, g], ref["slots"][r, g])
             assert misses[r, g] == ref["misses"][r, g]
-            assert np.max(np.abs(out[r, g] - ref["out"][r, g])) < ATTN_TOL
-            assert np.max(np.abs(lse[r, g] - ref["lse"][r, g])) < 1e-3
+        check_row_over_selection(idx[r, g], slots[r, g], misses[r, g], out[r, g], lse[r, g],
+                                 ref["q"][r, g], ref["K"][r, g], ref["V"][r, g],
+                                 ref["slot_map"][r, g], ref["hotK"][r, g], ref["hotV"][r, g], ke,
+                                 ref["scale"])
+    print(f"selection: {diff_rows} of {len(rows)} rows differ from the oracle inside the tie band "
+          f"({diffs} of {entries} entries)")
+    assert diffs <= max(2, max_diff_frac * entries)
     return diffs
 
 
@@ -249,16 +262,38 @@ def test_decode_step_ragged_batch(kvs, B):
 
 
 def test_decode_step_layer_sharing_reuses_selection(kvs):
-    """idx_in: the second layer of a group reads the first layer's selection."""
+    """idx_in: the second layer of a group reads the first layer's selection
+    ("MiniMax-M3: share the sparse index top-k across layers", description).
+    Layer 1 selects; layer 2 has its own queries, K/V caches and hot buffers
+    (built around that selection at 20% misses) and attends over the same
+    selection. Layer 2's slots, misses and attention are checked against the
+    oracle's gather and attention over layer 1's selection in layer 2's
+    caches; the selection buffer is not written by the reusing call."""
+    R, G, H, n_max, k, S = 2, 2, 4, 6000, 512, 1024
     nl = [6000, 5000]
-    ref, step = _decode_case(kvs, 2, 2, 4, nl, 6000, 92, 512, 1024, seed=3)
-    out1 = step.out.clone()
-    idx = step.idx.clone()
-    step.idx.fill_(-7)
-    step(step_q := synth.queries(2, 2, 4, D, seed=3).to(DEV), idx_in=idx)
+    ref, step = _decode_case(kvs, R, G, H, nl, n_max, 92, k, S, seed=3)
+    _check_decode(ref, step, R, G, nl, k)
+    idx1 = step.idx.clone()
+    K2, V2, _ = synth.fathom_kv(R, G, D, nl, n_max=n_max, seed=3, layer=1)
+    q2 = synth.queries(R, G, H, D, seed=3, layer=1)
+    sel = idx1.cpu().numpy()
+    slot_map2, hot_tok2 = synth.slot_map_from_selection(sel, nl, n_max, S, 0.2, seed=4)
+    hotK2, hotV2 = synth.hot_rows(K2, hot_tok2), synth.hot_rows(V2, hot_tok2)
+    ix2 = kvs.build_fathom_index(K2.to(DEV), nl)  # not read when a selection is given
+    step2 = kvs.DecodeStep(ix2, nl, n_max, H, 92, k, K2.to(DEV), V2.to(DEV),
+                           torch.from_numpy(slot_map2).to(DEV), hotK2.to(DEV), hotV2.to(DEV))
+    step2.idx.fill_(-7)
+    step2(q2.to(DEV), idx_in=idx1)
     torch.cuda.synchronize()
-    assert torch.all(step.idx == -7)  # not written when a selection is given
-    assert torch.equal(step.out, out1)
+    assert torch.all(step2.idx == -7)  # not written when a selection is given
+    for r in range(R):
+        for g in range(G):
+            ke = min(k, nl[r])
+            check_row_over_selection(sel[r, g], _np(step2.slots)[r, g], _np(step2.misses)[r, g],
+                                     _np(step2.out)[r, g], _np(step2.lse)[r, g], q2[r, g],
+                                     K2[r, g], V2[r, g], slot_map2[r, g], hotK2[r, g],
+                                     hotV2[r, g], ke, 1 / math.sqrt(D))
+            assert int(step2.misses[r, g]) == round(0.2 * ke)
 
 
 def test_decode_step_all_scores_tied_takes_first_indices(kvs):
@@ -358,7 +393,12 @@ def test_host_mapped_index_scan_and_decode(kvs, B):
             t, qbar = oracle.plan_bits(q[r, g], kvar[r, g], B)
             tol = fathom_score_tol(qbar, kmin[r, g], kstep[r, g], B)
             assert np.max(np.abs(sc[r, g] - ref["scores"][r, g])) <= tol
-            check_selection(step.idx[r, g].cpu().numpy(), ref["idx"][r, g], ref["scores"][r, g], 512)
+            gi = step.idx[r, g].cpu().numpy()
+            check_selection(gi, ref["idx"][r, g], ref["scores"][r, g], 512)
+            # no hot buffer: every selected row is read from the full store
+            check_row_over_selection(gi, None, _np(step.misses)[r, g], _np(step.out)[r, g],
+                                     _np(step.lse)[r, g], q[r, g], K[r, g], V[r, g], None, None,
+                                     None, min(512, nl[r]), 1 / math.sqrt(D))
 
 
 def test_decode_step_timed_matches_and_records_stages(kvs):

@@ -17,7 +17,7 @@ import torch
 
 import oracle
 import synth
-from tests._parity import ATTN_TOL, check_selection
+from tests._parity import check_row_over_selection, check_selection
 
 pytestmark = pytest.mark.gpu
 D, H = 128, 4
@@ -55,13 +55,14 @@ def _run_sampled(kvs, R, G, n, B, k, S, rows, seed):
                                   Vr, scale, want_scores=True)
         sel[r, g] = res["idx"][0, 0]
         ref[u] = dict(planes=planes[0, 0], kvar=kvar[0, 0], t=res["t"][0, 0], idx=res["idx"][0, 0],
-                      scores=res["scores"][0, 0], K=Kr, V=Vr, q=qr, index=(planes, kmin, kstep, kvar))
+                      scores=res["scores"][0, 0], K=Kr[0, 0], V=Vr[0, 0], q=qr[0, 0])
     slot_map, hot_tok = synth.slot_map_from_selection(sel, nl, n, S, 0.2, seed=seed)
     hotK, hotV = synth.hot_rows(K, hot_tok), synth.hot_rows(V, hot_tok)
     ix = kvs.build_fathom_index(K, nl, W)
     step = kvs.DecodeStep(ix, nl, n, H, B, k, K, V, torch.from_numpy(slot_map).to(DEV), hotK, hotV)
     step(q)
     torch.cuda.synchronize()
+    diffs = diff_rows = 0
     for u in rows:
         r, g = divmod(u, G)
         e = ref[u]
@@ -69,23 +70,34 @@ def _run_sampled(kvs, R, G, n, B, k, S, rows, seed):
         assert np.array_equal(ix.planes[r, g].cpu().numpy().view(np.uint32), e["planes"])
         assert np.array_equal(ix.kvar[r, g].cpu().numpy(), e["kvar"])
         assert np.array_equal(step.plan.t[r, g].cpu().numpy(), e["t"])
-        d = check_selection(step.idx[r, g].cpu().numpy(), e["idx"], e["scores"], k)
-        # the oracle's attention and misses over the same slot map
-        planes, kmin, kstep, kvar = e["index"]
-        res = oracle.decode_batch(e["q"], planes, kmin, kstep, kvar, [n], B, k,
-                                  slot_map[r, g][None, None], hotK[r, g].cpu()[None, None],
-                                  hotV[r, g].cpu()[None, None], e["K"], e["V"], scale)
+        gi = step.idx[r, g].cpu().numpy()
+        d = check_selection(gi, e["idx"], e["scores"], k)
+        diffs += d
+        diff_rows += d > 0
+        # slots, misses and attention: the oracle's gather and attention over
+        # the GPU's own selection, through the same slot map and hot rows
+        check_row_over_selection(gi, step.slots[r, g].cpu().numpy(), step.misses[r, g].item(),
+                                 step.out[r, g].cpu().numpy(), step.lse[r, g].cpu().numpy(),
+                                 e["q"], e["K"], e["V"], slot_map[r, g], hotK[r, g].cpu(),
+                                 hotV[r, g].cpu(), k, scale)
         if d == 0:
-            assert np.array_equal(step.slots[r, g].cpu().numpy(), res["slots"][0, 0])
-            assert int(step.misses[r, g]) == int(res["misses"][0, 0]) == round(0.2 * k)
-            assert np.max(np.abs(step.out[r, g].cpu().numpy() - res["out"][0, 0])) < ATTN_TOL
+            assert int(step.misses[r, g]) == round(0.2 * k)
+    print(f"selection: {diff_rows} of {len(rows)} sampled rows differ from the oracle inside the "
+          f"tie band ({diffs} of {len(rows) * k} entries)")
+    assert diffs <= max(2, 1e-3 * len(rows) * k)
+
+
+# 16 of the 128 rows of the 128K layer and 8 of the 32 rows of the 1M layer,
+# spread over the requests and heads, always with the last request's last head
+ROWS_128K = [0, 1, 9, 18, 27, 37, 46, 55, 64, 73, 82, 91, 100, 109, 118, 127]
+ROWS_1M = [0, 5, 9, 14, 18, 23, 27, 31]
 
 
 @pytest.mark.parametrize("B", [92, 68, 136, 512])
 def test_decode_step_128k_layer_sampled_rows(kvs, B):
-    _run_sampled(kvs, 16, 8, 131072, B, 2048, 4096, rows=[0, 37, 127], seed=100 + B)
+    _run_sampled(kvs, 16, 8, 131072, B, 2048, 4096, rows=ROWS_128K, seed=100 + B)
 
 
 @pytest.mark.parametrize("B", [92, 136])
 def test_decode_step_1m_layer_sampled_rows(kvs, B):
-    _run_sampled(kvs, 4, 8, 1048576, B, 2048, 4096, rows=[5, 31], seed=200 + B)
+    _run_sampled(kvs, 4, 8, 1048576, B, 2048, 4096, rows=ROWS_1M, seed=200 + B)

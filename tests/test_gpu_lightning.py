@@ -88,3 +88,65 @@ def test_lightning_layer_pair_block_topk_and_shared_attention(kvs):
         out_ref, lse_ref = oracle.shared_attention_batch(q.float(), K, V, idx.cpu().numpy(), scale)
         assert np.max(np.abs(step.out.cpu().numpy() - out_ref)) < ATTN_TOL
         assert np.all(step.misses.cpu().numpy() == k)
+
+
+def _check_block_selection(g_idx, o_idx, s_blocks, block):
+    """The GPU's block selection equals the oracle's, or differs only on blocks
+    whose oracle score lies within 1e-4 max|S| of the oracle's last selected
+    block. Returns the number of differing blocks."""
+    g_blocks = np.unique(g_idx[g_idx >= 0] // block)
+    o_blocks = np.unique(o_idx[o_idx >= 0] // block)
+    assert g_blocks.size == o_blocks.size
+    if np.array_equal(g_blocks, o_blocks):
+        return 0
+    kth = np.min(s_blocks[o_blocks])
+    tol = 1e-4 * np.max(np.abs(s_blocks[np.isfinite(s_blocks)]))
+    extra, missing = np.setdiff1d(g_blocks, o_blocks), np.setdiff1d(o_blocks, g_blocks)
+    assert np.all(s_blocks[extra] >= kth - tol)
+    assert np.all(s_blocks[missing] <= kth + tol)
+    return int(extra.size)
+
+
+def _lightning_vs_oracle(kvs, R, nl, n_max, Hi, block, k, reqs, seed):
+    kidx, qidx, w, _ = synth.lightning_inputs(R, nl, Hi=Hi, n_max=n_max, seed=seed, device=DEV)
+    bs = kvs.index_scan_lightning(kidx, qidx, w, nl, block=block)
+    idx = kvs.topk_select(bs, nl, k, block=block)
+    torch.cuda.synchronize()
+    bs, idx = bs.cpu().numpy(), idx.cpu().numpy()
+    sub = torch.tensor(reqs, dtype=torch.long, device=DEV)
+    ref_bs, ref_idx = oracle.lightning_batch(kidx[sub].cpu(), qidx[sub].cpu(), w[sub].cpu(),
+                                             [nl[r] for r in reqs], block, k)
+    diffs = 0
+    for j, r in enumerate(reqs):
+        nbr = (nl[r] + block - 1) // block
+        if nbr:
+            ref = ref_bs[j, :nbr]
+            tol = 1e-4 * max(1e-30, float(np.max(np.abs(ref))))
+            err = float(np.max(np.abs(bs[r, :nbr] - ref)))
+            assert err <= tol, (r, err, tol)
+        assert np.all(np.isneginf(bs[r, nbr:]))
+        diffs += _check_block_selection(idx[r], ref_idx[j], ref_bs[j, :nbr], block)
+    print(f"block selection: {diffs} blocks differ from the oracle inside the tie band over "
+          f"{len(reqs)} requests")
+    return diffs
+
+
+def test_lightning_full_size_sampled_requests(kvs):
+    """The lightning layer at its full size (32 requests x 80000 tokens, 64
+    index heads, 64-token blocks, top-2048 tokens): every block of the kernel's
+    grid runs about 135 tiles, so its raw-tile and accumulator rings wrap many
+    times. Four sampled requests (the last one included) against the oracle."""
+    R, n = 32, 80000
+    _lightning_vs_oracle(kvs, R, [n] * R, n, 64, 64, 2048, reqs=[0, 9, 22, 31], seed=5)
+
+
+def test_lightning_many_short_requests_cross_boundaries(kvs):
+    """600 requests of at most 384 tokens (ragged, some empty): about 12 tiles
+    per block of the grid, each block crossing three or more request
+    boundaries, so the query buffers, head-weight slots and rings all rotate.
+    Every request against the oracle."""
+    R, n_max = 600, 384
+    rng = np.random.default_rng(11)
+    nl = [int(x) for x in rng.integers(1, n_max + 1, size=R)]
+    nl[0], nl[17], nl[599], nl[300] = n_max, 0, n_max, 1
+    _lightning_vs_oracle(kvs, R, nl, n_max, 64, 64, 128, reqs=list(range(R)), seed=6)

@@ -418,3 +418,79 @@ def test_decode_batch_composes_the_steps():
             out, lse = oracle.attention(q[r, g], K[r, g][idx], V[r, g][idx], k_eff, 1 / math.sqrt(D))
             assert np.array_equal(out, res["out"][r, g])
             assert res["misses"][r, g] == k_eff  # no hot buffer: every row is a miss
+
+
+def _lightning_numpy(kidx, qidx, w, nr, block, k):
+    """Lightning selection for one request written out with numpy/torch alone:
+    e4m3 and bf16 decoded by torch, S = relu(K Q^T) w in fp64, block max over
+    the valid tokens, top (k / block) blocks by (score desc, block asc)."""
+    kf = kidx[:nr].view(torch.float8_e4m3fn).double().numpy()
+    qf = qidx.double().numpy()
+    s = np.maximum(0.0, kf @ qf.T) @ w.double().numpy()
+    nb = (nr + block - 1) // block
+    pad = np.full(nb * block, -np.inf)
+    pad[:nr] = s
+    bm = pad.reshape(nb, block).max(axis=1) if nb else np.zeros(0)
+    order = np.lexsort((np.arange(nb), -bm))[: k // block]
+    toks = [np.arange(b * block, min(nr, (b + 1) * block)) for b in np.sort(order)]
+    idx = np.full(k, -1, np.int64)
+    if toks:
+        t = np.concatenate(toks)
+        idx[: t.size] = t
+    return bm, idx
+
+
+def test_lightning_batch_is_the_per_request_selection():
+    """Every request of the batch driver equals the selection written out with
+    numpy on that request's own slices (ragged lengths, different data per
+    request), and a request subset fills only its own rows."""
+    nl = [700, 333, 320, 0, 65]
+    R, Hi, block, k = len(nl), 16, 64, 256
+    kidx, qidx, w, _ = synth.lightning_inputs(R, nl, Hi=Hi, n_max=700, seed=17)
+    bs, idx = oracle.lightning_batch(kidx, qidx, w, nl, block, k)
+    nbmax = (700 + block - 1) // block
+    assert bs.shape == (R, nbmax) and idx.shape == (R, k)
+    for r in range(R):
+        bm, ref = _lightning_numpy(kidx[r], qidx[r], w[r], nl[r], block, k)
+        nb = bm.size
+        assert np.allclose(bs[r, :nb], bm, rtol=1e-12, atol=0)
+        assert np.all(np.isneginf(bs[r, nb:]))
+        assert np.array_equal(idx[r], ref), r
+    # the same requests through the subset argument, in another order
+    bs2, idx2 = oracle.lightning_batch(kidx, qidx, w, nl, block, k, reqs=[2, 0])
+    assert np.array_equal(bs2[[0, 2]], bs[[0, 2]]) and np.array_equal(idx2[[0, 2]], idx[[0, 2]])
+    assert not idx2[[1, 3, 4]].any() and not bs2[[1, 3, 4]].any()
+
+
+def test_shared_attention_batch_reads_each_requests_selection():
+    """Every (request, KV head) row attends, with numpy's dense softmax, over
+    the rows that request's own selection names in that head's own K/V
+    (different selections per request, -1 padding skipped); a row subset fills
+    only its rows."""
+    R, G, H, n_max, k = 3, 2, 4, 500, 64
+    K, V, _ = synth.fathom_kv(R, G, D, [500, 410, 77], n_max=n_max, seed=29)
+    q = synth.queries(R, G, H, D, seed=29)
+    rng = np.random.default_rng(29)
+    idx = np.full((R, k), -1, np.int32)
+    for r, (kk, hi) in enumerate([(64, 500), (50, 410), (9, 77)]):
+        idx[r, :kk] = np.sort(rng.choice(hi, kk, replace=False))
+    scale = 1 / math.sqrt(D)
+    out, lse = oracle.shared_attention_batch(q, K, V, idx, scale)
+    for r in range(R):
+        sel = idx[r][idx[r] >= 0]
+        for g in range(G):
+            Kf, Vf = _bf16_np(K[r, g])[sel], _bf16_np(V[r, g])[sel]
+            logits = (q[r, g].double().numpy() @ Kf.T) * scale
+            mx = logits.max(axis=1, keepdims=True)
+            p = np.exp(logits - mx)
+            assert np.allclose(out[r, g], (p / p.sum(axis=1, keepdims=True)) @ Vf, rtol=1e-12,
+                               atol=1e-13)
+            assert np.allclose(lse[r, g], mx[:, 0] + np.log(p.sum(axis=1)), rtol=1e-13)
+    rows = [5, 0]  # (r=2, g=1) and (r=0, g=0)
+    out2, lse2 = oracle.shared_attention_batch(q, K, V, idx, scale, rows=rows)
+    for u in range(R * G):
+        r, g = divmod(u, G)
+        if u in rows:
+            assert np.array_equal(out2[r, g], out[r, g]) and np.array_equal(lse2[r, g], lse[r, g])
+        else:
+            assert not out2[r, g].any()

@@ -55,18 +55,38 @@ def test_noalloc_matches_workspace_attention_on_two_calls_in_a_row(kvs):
         outs.append(out)
 
 
-def test_noalloc_rejects_sizes_beyond_its_array(kvs):
-    H, k, G = 8, 2048, 4
-    sizes = [R for R in range(1, 400)
-             if kvs._lib.kvs_attn_workspace_size(R, G, H, k) > 4 << 20]
-    if not sizes:
-        pytest.skip("no size needs more than the fixed array on this GPU")
-    R = sizes[0]
-    q = torch.zeros(R, G, H, D, device="cuda")
-    K = torch.zeros(R, G, 8, D, dtype=torch.bfloat16, device="cuda")
-    out = torch.empty(R, G, H, D, device="cuda")
-    st = kvs._lib.sparse_decode_attn_noalloc(q.data_ptr(), 0, K.data_ptr(), K.data_ptr(), None, R,
-                                             G, H, D, k, 0.1, out.data_ptr(), None, None,
-                                             torch.cuda.current_stream().cuda_stream)
-    assert st == kvs.KVS_EINVAL
-    assert b"fixed" in kvs._lib.kvs_last_error()
+def test_noalloc_sizes_beyond_the_workspace_split_run_with_fewer_splits(kvs):
+    """At H = 4, k = 2048 the workspace attention cuts the rows of 593 and 2073
+    (request, KV head) pairs into splits whose partial results need more than
+    the fixed 4 MiB array (7.2 and 8.8 MiB on a 148-SM B200). The no-allocation
+    call runs them with fewer splits, and matches, twice in a row."""
+    H, k, G = 4, 2048, 1
+    for RG in (593, 2073):
+        assert kvs._lib.kvs_attn_workspace_size(RG, G, H, k) > 4 << 20
+        q, K, V, k_eff = _case(RG, RG, G, H, k, torch.float32)
+        ref_out, ref_lse = kvs.sparse_decode_attn(q, K, V, k_eff=k_eff)
+        for _ in range(2):
+            out = torch.full((RG, G, H, D), float("nan"), device="cuda")
+            lse = torch.full((RG, G, H), float("nan"), device="cuda")
+            kvs.sparse_decode_attn_noalloc(q, K, V, out, lse, k_eff=k_eff)
+            torch.cuda.synchronize()
+            assert float((out - ref_out).abs().max()) < ATTN_TOL
+            fin = torch.isfinite(ref_lse)
+            assert torch.equal(fin, torch.isfinite(lse))
+            assert float((lse[fin] - ref_lse[fin]).abs().max()) < 1e-3
+
+
+def test_noalloc_checks_caller_outputs(kvs):
+    """The binding refuses output buffers that the kernels would overrun."""
+    q, K, V, k_eff = _case(13, 2, 3, 4, 64, torch.float32)
+    bad = [torch.empty(2, 3, 4, D, dtype=torch.bfloat16, device="cuda"),
+           torch.empty(2, 3, 4, D + 1, device="cuda")[..., :D],
+           torch.empty(2, 3, 3, D, device="cuda")]
+    for out in bad:
+        with pytest.raises(ValueError):
+            kvs.sparse_decode_attn_noalloc(q, K, V, out)
+    out = torch.empty(2, 3, 4, D, device="cuda")
+    with pytest.raises(ValueError):
+        kvs.sparse_decode_attn_noalloc(q, K, V, out, torch.empty(2, 3, 5, device="cuda"))
+    with pytest.raises(ValueError):
+        kvs.sparse_decode_attn_noalloc(q, K, V, out, k_eff=k_eff.long())
