@@ -1,6 +1,6 @@
 """Benchmark of the per-step top-k sparse-attention decode path on B200.
 
-Default workload (one GPU): the Qwen3-8B-shaped 128K decode layer -- 16
+Headline workload (one GPU): the Qwen3-8B-shaped 128K decode layer -- 16
 requests, 8 KV heads of 4 query heads, d = 128, 131072 keys each, a 92-bit
 Fathom budget per key, top-2048 per (request, KV head), a 4096-entry hot
 buffer per (request, KV head) holding 80% of the selection. One step is one
@@ -10,8 +10,24 @@ slot lookup and sparse GQA attention.
 metric: keys scored per second by the full decode step (each step scores
 R*G*n keys); layer-steps/s and achieved HBM GB/s are reported beside it.
 Inputs are synthetic (seeded draws with the pages' shapes and distributions)
-and stay resident in HBM; every step reads ~350 MB, more than the 126 MB L2,
-so no L2 flush is needed between steps.
+and stay resident in HBM; every step reads more than the 126 MB L2, so no L2
+flush is needed between steps.
+
+The same JSON line carries, under "configs", one entry per other measured
+workload, each timed with the same --steps/--warmup and each with its own
+roofline (algorithmic bytes of its dominant kernel / that kernel's CUDA-event
+time / the measured peak) and a short CPU-oracle sample:
+  128k-B68, 128k-B136, 128k-B512  the 128K layer at the other budgets;
+  1m-B92, 1m-B136                 the 1M layer (4 x 8 x 1048576), index in HBM;
+  1m-host-B92                     the 1M layer with the index planes in mapped
+                                  pinned host memory, read by the scan over
+                                  the host link (roofline: a pinned
+                                  host-to-device copy measured in the run);
+  lightning-pair                  32 requests x 80000 tokens: lightning
+                                  indexer (64 heads, tcgen05), block top-k,
+                                  and sparse attention for both layers of a
+                                  group reusing one selection.
+--only-headline skips them.
 
 --impl reference times the CPU oracle (the only reference this method has) on
 a bounded sample of the same workload, on the host cores.
@@ -25,9 +41,8 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
+import threading
 import time
 
 import numpy as np
@@ -44,19 +59,18 @@ WORKLOADS = {
     "qwen3-8b-1m": dict(R=4, G=8, H=4, n=1048576, B=92, k=2048, S=4096, miss=0.2),
     "tiny": dict(R=1, G=1, H=4, n=4096, B=92, k=256, S=512, miss=0.2),
 }
+LIGHTNING = dict(R=32, n=80000, Hi=64, Dl=128, block=64, k=2048, G=8, H=4)
 METRIC = "index-scan keys/s + sparse decode layer-steps/s; achieved GB/s vs HBM peak"
-# the dominant kernel of a step with a plan of <= 144 planes: the byte-indexed
-# scan, which reads the plan's planes and writes every score and 16-key maximum
-SCAN_KERNEL = "fathom_scan_prmt (scan stage of the step)"
 
-# DRAM bytes (read + write) of one launch of the fused scan + top-k kernel, from
-# ncu captures of a smaller case of the same workload scaled to a full launch by
+# DRAM bytes (read + write) of one launch of the scan kernel, from ncu
+# captures of a smaller case of the same workload scaled to a full launch by
 # the keys processed (the capture and scaling are stated under profiles/);
-# None where no capture of the current kernel exists.
+# keyed by (workload, B, kernel). Absent where no capture of the current kernel
+# exists.
 TRAFFIC: dict = {
     # R=8 capture of fathom_scan_prmt_kernel: 96.56 MB read + 9.77 MB written
     # per launch (the rest of its scores leave L2 later), x2 for R=16
-    ("qwen3-8b-128k", 92): 2 * (96_558_080 + 9_770_752),
+    ("qwen3-8b-128k", 92, "fathom_scan_prmt"): 2 * (96_558_080 + 9_770_752),
 }
 
 
@@ -65,8 +79,8 @@ def _peaks():
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    return 6650.0, "fallback"
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", 1590.0)), "measured"
+    return 6650.0, 1590.0, "fallback"
 
 
 def _dist():
@@ -93,21 +107,21 @@ def _max_over_ranks(dist, x: float) -> float:
 
 
 class Clocks:
-    """SM clock and throttle-reason samples taken every 10 ms by an NVML thread
-    while the timed region runs (nvidia-smi is the fallback). The sampler is
-    started before the region and must have one sample under load before the
-    region starts."""
+    """SM clock and throttle-reason samples from an NVML thread, about every
+    0.2 ms for as long as the benchmark runs GPU work. Each timed region is
+    marked by host timestamps taken just before its first launch and just
+    after its closing synchronize; a region's clock record is the samples that
+    fall inside it (the headline region of 20 steps lasts a few ms)."""
 
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4}
 
     def __init__(self):
-        self.samples = []
-        self.reasons = set()
+        self.samples = []  # (host time, sm MHz, reason bits)
         self.max_mhz = None
+        self.error = None
         self._stop = False
         self._thread = None
-        self._nvml = None
 
     def _handle(self):
         import pynvml
@@ -125,166 +139,245 @@ class Clocks:
         return pynvml, pynvml.nvmlDeviceGetHandleByIndex(idx)
 
     def start(self):
-        import threading
         try:
             nv, h = self._handle()
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
         except Exception as e:  # no NVML
-            self.reasons.add(f"nvml unavailable: {type(e).__name__}")
+            self.error = f"nvml unavailable: {type(e).__name__}"
             return
-        self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        reasons_fn = (nv.nvmlDeviceGetCurrentClocksEventReasons
+                      if hasattr(nv, "nvmlDeviceGetCurrentClocksEventReasons")
+                      else nv.nvmlDeviceGetCurrentClocksThrottleReasons)
 
         def loop():
             while not self._stop:
                 try:
-                    self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
-                    r = (nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                         if hasattr(nv, "nvmlDeviceGetCurrentClocksEventReasons")
-                         else nv.nvmlDeviceGetCurrentClocksThrottleReasons(h))
-                    for name, bit in self.REASONS.items():
-                        if r & bit:
-                            self.reasons.add(name)
+                    mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    self.samples.append((time.perf_counter(), mhz, int(reasons_fn(h))))
                 except Exception:
                     pass
-                time.sleep(0.01)
+                time.sleep(0.0002)
 
         self._thread = threading.Thread(target=loop, daemon=True)
         self._thread.start()
-
-    def wait_first(self, timeout=2.0):
         t0 = time.time()
-        while self._thread is not None and not self.samples and time.time() - t0 < timeout:
-            time.sleep(0.005)
-        self.samples.clear()
+        while not self.samples and time.time() - t0 < 2.0:
+            time.sleep(0.001)
 
-    def stop(self) -> dict:
+    def stop(self):
         self._stop = True
         if self._thread is not None:
             self._thread.join()
-        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
-                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                "samples": len(self.samples)}
+
+    def window(self, t0: float, t1: float) -> dict:
+        s = [x for x in self.samples if t0 <= x[0] <= t1]
+        reasons = sorted({name for _, _, r in s for name, bit in self.REASONS.items() if r & bit})
+        out = {"sm_mhz": statistics.median([m for _, m, _ in s]) if s else None,
+               "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(s)}
+        if self.error:
+            out["error"] = self.error
+        return out
 
 
-def setup(cfg: dict, device, seed: int = 1):
-    """Synthetic inputs resident on the device, a warm-up selection, and the hot
-    buffers built around it (80% of the selected rows present)."""
+CLOCKS = Clocks()
+
+
+class Region:
+    """Host timestamps around a timed region (for the clock record)."""
+
+    def __enter__(self):
+        self.t0 = time.perf_counter()
+        return self
+
+    def __exit__(self, *a):
+        self.t1 = time.perf_counter()
+
+    def clocks(self) -> dict:
+        return CLOCKS.window(self.t0, self.t1)
+
+
+# ----------------------------------------------------------------------------- Fathom decode step
+
+def setup_fathom(cfg: dict, device, seed: int = 1, host_index: bool = False):
+    """Synthetic caches, queries and the index resident on the device."""
     import kv_index_scan_b200 as kvs
-    R, G, H, n, B, k, S = (cfg[x] for x in ("R", "G", "H", "n", "B", "k", "S"))
+    R, G, H, n = (cfg[x] for x in ("R", "G", "H", "n"))
     K, V, nl = synth.fathom_kv(R, G, 128, n, seed=seed, device=device)
     q = synth.queries(R, G, H, 128, seed=seed, device=device)
     index = kvs.build_fathom_index(K, nl)
-    warm = kvs.DecodeStep(index, nl, n, H, B, k, K, V)
-    warm(q)
+    return dict(K=K, V=V, q=q, index=index, nl=nl, seed=seed)
+
+
+def decode_step_for(cfg: dict, data: dict, B: int, index=None):
+    """A DecodeStep at budget B with hot buffers built around a warm-up
+    selection of that budget (cfg['miss'] of each selection missing)."""
+    import kv_index_scan_b200 as kvs
+    R, G, H, n, k, S = (cfg[x] for x in ("R", "G", "H", "n", "k", "S"))
+    index = index or data["index"]
+    warm = kvs.DecodeStep(index, data["nl"], n, H, B, k, data["K"], data["V"])
+    warm(data["q"])
     torch.cuda.synchronize()
     sel = warm.idx.cpu().numpy()
     del warm
-    slot_map, hot_tok = synth.slot_map_from_selection(sel, nl, n, S, cfg["miss"], seed=seed)
-    hotK, hotV = synth.hot_rows(K, hot_tok), synth.hot_rows(V, hot_tok)
-    slot_map_t = torch.from_numpy(slot_map).to(device)
-    step = kvs.DecodeStep(index, nl, n, H, B, k, K, V, slot_map_t, hotK, hotV)
-    return dict(K=K, V=V, q=q, index=index, step=step, nl=nl, slot_map=slot_map_t, hotK=hotK,
-                hotV=hotV, sel=sel)
+    slot_map, hot_tok = synth.slot_map_from_selection(sel, data["nl"], n, S, cfg["miss"],
+                                                      seed=data["seed"])
+    hotK, hotV = synth.hot_rows(data["K"], hot_tok), synth.hot_rows(data["V"], hot_tok)
+    slot_map_t = torch.from_numpy(slot_map).to(data["K"].device)
+    step = kvs.DecodeStep(index, data["nl"], n, H, B, k, data["K"], data["V"], slot_map_t, hotK,
+                          hotV)
+    return step, dict(slot_map=slot_map_t, hotK=hotK, hotV=hotV)
 
 
-def algorithmic_bytes(cfg: dict) -> dict:
-    R, G, n, B, k = (cfg[x] for x in ("R", "G", "n", "B", "k"))
+def algorithmic_bytes(cfg: dict, B: int) -> dict:
+    R, G, n, k = (cfg[x] for x in ("R", "G", "n", "k"))
     keys = R * G * n
     scan = keys * B / 8
     rows = R * G * k * (2 * 128 * 2 + 32)  # K + V rows and one 32-byte slot-map sector
     return dict(keys=keys, scan=scan, rows=rows, total=scan + rows)
 
 
-def time_steps(fn, steps: int, warmup: int, stream) -> float:
-    for _ in range(warmup):
-        fn()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        fn()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / steps
+def scan_kernel_name(B: int, host: bool) -> str:
+    if host:
+        return "fathom_scan_simple"
+    return "fathom_scan_prmt" if B <= 144 else "fathom_scan_topk"
 
 
-def run_ours(args, cfg, dist, rank, ws):
-    import kv_index_scan_b200 as kvs
-    dev = torch.device("cuda", torch.cuda.current_device())
-    data = setup(cfg, dev, seed=1 + rank)
-    step, q = data["step"], data["q"]
+def time_decode_steps(step, q, steps: int, warmup: int, dist=None):
+    """Warm-up, then exactly `steps` decode steps between CUDA events on the
+    launching stream. Every 8th timed step runs decode_step_timed, whose events
+    bracket each stage on the same stream, so the dominant kernel's duration is
+    measured inside the timed region. Returns (ms per step, stage ms, region)."""
     stream = torch.cuda.current_stream()
-    algo = algorithmic_bytes(cfg)
-
-    # ---- device-resident timed region: whole decode steps ----
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step(q)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    # every 8th step records its stage boundaries (decode_step_timed), so the
-    # dominant kernel's launch duration is measured inside the timed region at
-    # a negligible cost to the others
     nst = len(step.DECODE_STAGES)
-    every = 8
-    timed_steps = list(range(0, args.steps, every))
+    timed_steps = list(range(0, steps, 8))
     ev = {i: [torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for i in timed_steps}
-    clocks = Clocks()
-    clocks.start()
-    clocks.wait_first()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.steps):
-        if i in ev:
-            step.timed(q, ev[i])
-        else:
-            step(q)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.steps
-    clk = clocks.stop()
-    stages_ms = {name: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in timed_steps) / len(timed_steps)
-                 for j, name in enumerate(step.DECODE_STAGES)}
-    if dist:
-        dist.barrier()
-    ms_max = _max_over_ranks(dist, ms)
-    if args.only_step:
-        if rank == 0:
-            print(json.dumps({"ms_per_step": ms_max, "stages_ms": stages_ms}), flush=True)
-        return None
+    with Region() as reg:
+        e0.record(stream)
+        for i in range(steps):
+            if i in ev:
+                step.timed(q, ev[i])
+            else:
+                step(q)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    stages = {name: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in timed_steps) / len(timed_steps)
+              for j, name in enumerate(step.DECODE_STAGES)}
+    return ms, stages, reg
 
-    # ---- the bit-plane scan alone (scores to HBM, no top-k), same stream ----
-    scan_scores = torch.empty(cfg["R"], cfg["G"], cfg["n"], dtype=torch.float32, device=dev)
-    plan = step.plan
 
-    def scan_once():
-        kvs.index_scan_fathom(data["index"], plan, step.n, cfg["n"], scores=scan_scores)
+def oracle_sample(cfg, data, B, hot, rows: int, min_seconds: float) -> dict:
+    """The CPU oracle, as it stands, on a bounded sample of the workload:
+    `rows` (request, KV head) rows of one decode step, all host cores."""
+    import oracle
+    R, G, n, k = (cfg[x] for x in ("R", "G", "n", "k"))
+    rows = min(rows, R * G)
+    us = list(range(rows))
+    rr = [u // G for u in us]
+    gg = [u % G for u in us]
+    K = data["K"][rr, gg].unsqueeze(0).cpu()
+    V = data["V"][rr, gg].unsqueeze(0).cpu()
+    q = data["q"][rr, gg].unsqueeze(0).cpu()
+    nl = [data["nl"][0]]
+    sm = hot["slot_map"][rr, gg].unsqueeze(0).cpu()
+    hK = hot["hotK"][rr, gg].unsqueeze(0).cpu()
+    hV = hot["hotV"][rr, gg].unsqueeze(0).cpu()
+    W = synth.plane_words(n)
+    planes, kmin, kstep, kvar = oracle.build_index_batch(K, nl, W)  # data prep, not timed
+    cores = os.cpu_count() or 1
+    reps, t0 = 0, time.perf_counter()
+    while True:  # repeat the bounded sample for about min_seconds of CPU work
+        oracle.decode_batch(q, planes, kmin, kstep, kvar, nl, B, k, sm, hK, hV, K, V,
+                            1 / math.sqrt(128), nthreads=cores)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_seconds or reps >= 5000:
+            break
+    return {"value": reps * rows * n / dt, "unit": "keys/s", "cores": cores, "kind": "oracle",
+            "sample": f"{rows} of {R * G} (request, KV head) rows of one decode step "
+                      f"({rows * n} keys) x {reps} repetitions, fp64 C++ oracle on {cores} "
+                      f"threads, {dt:.1f} s"}
 
-    scan_ms = time_steps(scan_once, max(args.steps, 5), 3, stream)
 
-    # ---- end to end through the C ABI with host buffers ----
-    # Every step copies its q from pinned host memory and its out, idx and
-    # misses back to pinned host memory. The copies run on two copy streams
-    # (the copy engines) beside the compute stream: step i's results are read
-    # back while step i + 1 computes, into the other of two output sets (two
-    # DecodeSteps over the same index and caches).
-    R, G, H = cfg["R"], cfg["G"], cfg["H"]
-    step_b = kvs.DecodeStep(data["index"], data["nl"], cfg["n"], H, cfg["B"], cfg["k"], data["K"],
-                            data["V"], data["slot_map"], data["hotK"], data["hotV"])
+def decode_entry(name, cfg, data, B, args, dist, ws, peak, peak_kind, cpu_rows, cpu_seconds,
+                 host_index=None, link_peak=None):
+    """One decode-step measurement at budget B: throughput, stage times, the
+    scan's roofline, and a CPU-oracle sample (rank 0)."""
+    step, hot = decode_step_for(cfg, data, B, index=host_index)
+    ms, stages, reg = time_decode_steps(step, data["q"], args.steps, args.warmup, dist)
+    ms = _max_over_ranks(dist, ms)
+    algo = algorithmic_bytes(cfg, B)
+    kern = scan_kernel_name(B, host_index is not None)
+    scan_gbs = algo["scan"] / (stages["scan"] / 1e3) / 1e9
+    if host_index is not None:
+        roof = {"bound": "host-link", "kernel": kern + " (scan stage of the step, planes over the host link)",
+                "achieved": scan_gbs, "peak": link_peak, "peak_kind": "pinned host-to-device copy of the same bytes, measured in this run",
+                "unit": "GB/s", "frac": scan_gbs / link_peak, "traffic": None,
+                "algorithmic_bytes": algo["scan"], "ms": stages["scan"]}
+    else:
+        roof = {"bound": "hbm", "kernel": kern + " (scan stage of the step)", "achieved": scan_gbs,
+                "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": scan_gbs / peak,
+                "traffic": TRAFFIC.get((cfg["name"], B, kern)), "algorithmic_bytes": algo["scan"],
+                "ms": stages["scan"]}
+        if B <= 144:  # the scan also writes every score and 16-key maximum
+            roof["bytes_moved"] = algo["scan"] + algo["keys"] * (4 + 4 / 16)
+    R, G = cfg["R"], cfg["G"]
+    res = {"workload": cfg["name"], "bits_per_key": B, "requests": R, "kv_heads": G,
+           "context": cfg["n"], "topk": cfg["k"], "hot_slots": cfg["S"], "miss_rate": cfg["miss"],
+           "ms_per_step": ms, "keys_per_s": algo["keys"] * ws / (ms / 1e3),
+           "layer_steps_per_s": ws * 1e3 / ms,
+           "achieved_gbs": algo["total"] * ws / (ms / 1e3) / 1e9,
+           "step_frac_hbm": algo["total"] / (ms / 1e3) / 1e9 / peak,
+           "bytes_per_key": algo["scan"] / algo["keys"],
+           "miss_rate_measured": int(step.misses.sum().item()) / (R * G * cfg["k"]),
+           "stages_ms": stages, "roofline": roof, "clocks": reg.clocks(),
+           "index": "mapped pinned host memory" if host_index is not None else "hbm"}
+    if dist is None or dist.get_rank() == 0:
+        if cpu_rows > 0:
+            res["cpu_baseline"] = oracle_sample(cfg, data, B, hot, cpu_rows, cpu_seconds)
+    res["_step"], res["_hot"] = step, hot
+    return res
+
+
+def _strip(d: dict) -> dict:
+    return {k: v for k, v in d.items() if not k.startswith("_")}
+
+
+def e2e_entry(cfg, data, step, hot, args, dist, B):
+    """End to end through the C ABI with host buffers: every step copies its q
+    from pinned host memory and its out, idx and misses back to pinned host
+    memory. The copies run on two copy streams beside the compute stream: step
+    i's results are read back while step i + 1 computes, into the other of two
+    output sets (two DecodeSteps over the same index and caches). The timed
+    region ends when the last step's results are on the host."""
+    import kv_index_scan_b200 as kvs
+    R, G, H, k = cfg["R"], cfg["G"], cfg["H"], cfg["k"]
+    q = data["q"]
+    stream = torch.cuda.current_stream()
+    step_b = kvs.DecodeStep(data["index"], data["nl"], cfg["n"], H, B, k, data["K"], data["V"],
+                            hot["slot_map"], hot["hotK"], hot["hotV"])
     steps2 = (step, step_b)
     q_host = q.cpu().pin_memory()
     out_host = [torch.empty(R, G, H, 128, dtype=torch.float32).pin_memory() for _ in range(2)]
-    idx_host = [torch.empty(R, G, cfg["k"], dtype=torch.int32).pin_memory() for _ in range(2)]
+    idx_host = [torch.empty(R, G, k, dtype=torch.int32).pin_memory() for _ in range(2)]
     miss_host = [torch.empty(R, G, dtype=torch.int32).pin_memory() for _ in range(2)]
     q_devs = [torch.empty_like(q) for _ in range(2)]
     h2d_stream, d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
-    ev = lambda: torch.cuda.Event()
-    q_ready, done, copied = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    q_ready = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    copied = [torch.cuda.Event() for _ in range(2)]
     for b in range(2):  # every event exists before its first wait
         for e in (q_ready[b], done[b], copied[b]):
             e.record(stream)
 
-    def e2e_once(i):
+    def once(i):
         b = i & 1
         st = steps2[b]
         with torch.cuda.stream(h2d_stream):
@@ -302,62 +395,248 @@ def run_ours(args, cfg, dist, rank, ws):
             miss_host[b].copy_(st.misses, non_blocking=True)
             copied[b].record(d2h_stream)
 
-    def time_e2e(steps: int, warmup: int) -> float:
-        for i in range(warmup):
-            e2e_once(i)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(args.warmup):
+        once(i)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Region() as reg:
         e0.record(stream)
-        for i in range(steps):
-            e2e_once(i)
-        for b in range(2):  # the region ends when the last results are on the host
+        for i in range(args.steps):
+            once(i)
+        for b in range(2):
             stream.wait_event(copied[b])
         e1.record(stream)
         torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / steps
+    ms = _max_over_ranks(dist, e0.elapsed_time(e1) / args.steps)
+    last = (args.steps - 1) & 1
+    assert torch.equal(idx_host[last], steps2[last].idx.cpu())
+    h2d = q_host.numel() * q_host.element_size()
+    d2h = sum(t[0].numel() * t[0].element_size() for t in (out_host, idx_host, miss_host))
+    return ms, h2d, d2h, reg
 
-    e2e_ms = _max_over_ranks(dist, time_e2e(args.steps, args.warmup))
-    assert torch.equal(idx_host[(args.steps - 1) & 1], steps2[(args.steps - 1) & 1].idx.cpu())
-    q_host_bytes = q_host.numel() * 4
-    h2d = q_host_bytes
-    d2h = out_host[0].numel() * 4 + idx_host[0].numel() * 4 + miss_host[0].numel() * 4
-    misses = int(step.misses.sum().item())
 
-    peak, peak_kind = _peaks()
+def run_ours(args, dist, rank, ws):
+    import kv_index_scan_b200 as kvs
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peak, bf16_peak, peak_kind = _peaks()
+    CLOCKS.start()
+    stream = torch.cuda.current_stream()
+    cfg = dict(WORKLOADS[args.workload], name=args.workload)
+    if args.B is not None:
+        cfg["B"] = args.B
+    if args.requests is not None:
+        cfg["R"] = args.requests
+    B = cfg["B"]
+    data = setup_fathom(cfg, dev, seed=1 + rank)
+
+    # ---- headline: device-resident fused decode steps ----
+    head = decode_entry(args.workload, cfg, data, B, args, dist, ws, peak, peak_kind,
+                        0 if args.no_cpu_baseline else args.cpu_rows, 10.0)
+    step, hot = head["_step"], head["_hot"]
+    if args.only_step:
+        if rank == 0:
+            print(json.dumps({"ms_per_step": head["ms_per_step"], "stages_ms": head["stages_ms"]}),
+                  flush=True)
+        return None
+
+    # ---- the bit-plane scan alone (scores to HBM, no top-k), same stream ----
+    scan_scores = torch.empty(cfg["R"], cfg["G"], cfg["n"], dtype=torch.float32, device=dev)
+
+    def scan_once():
+        kvs.index_scan_fathom(data["index"], step.plan, step.n, cfg["n"], scores=scan_scores)
+
+    for _ in range(3):
+        scan_once()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    nscan = max(args.steps, 5)
+    e0.record(stream)
+    for _ in range(nscan):
+        scan_once()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    scan_ms = e0.elapsed_time(e1) / nscan
+    del scan_scores
+    algo = algorithmic_bytes(cfg, B)
+    scan_gbs = algo["scan"] / (scan_ms / 1e3) / 1e9
+
+    # ---- end to end through the C ABI with host buffers ----
+    e2e_ms, h2d, d2h, _ = e2e_entry(cfg, data, step, hot, args, dist, B)
+
     keys_total = algo["keys"] * ws
-    value = keys_total / (ms_max / 1e3)
-    scan_bytes = algo["scan"]
-    scan_gbs = scan_bytes / (scan_ms / 1e3) / 1e9
-    launches_per_step = 4 + (1 if step_needs_combine(cfg) else 0)  # plan, scan+top-k, merge, attention (+ split merge)
+    ms_max = head["ms_per_step"]
+    launches_per_step = 4 + (1 if step_needs_combine(cfg) else 0)  # plan, scan, top-k, attention (+ split merge)
     res = {
-        "metric": METRIC, "value": value, "unit": "keys/s", "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": args.workload, "requests": R, "kv_heads": G, "q_heads_per_kv": H,
-                   "head_dim": 128, "context": cfg["n"], "bits_per_key": cfg["B"],
-                   "topk": cfg["k"], "hot_slots": cfg["S"], "miss_rate": cfg["miss"],
+        "metric": METRIC, "value": keys_total / (ms_max / 1e3), "unit": "keys/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "requests": cfg["R"], "kv_heads": cfg["G"],
+                   "q_heads_per_kv": cfg["H"], "head_dim": 128, "context": cfg["n"],
+                   "bits_per_key": B, "topk": cfg["k"], "hot_slots": cfg["S"],
+                   "miss_rate": cfg["miss"],
                    "parallelism": f"replicas{ws}" if ws > 1 else "single",
                    "l2": "inputs larger than L2 (>=350 MB read per step)"},
-        "layer_steps_per_s": ws * 1e3 / ms_max,
-        "achieved_gbs": algo["total"] * ws / (ms_max / 1e3) / 1e9,
-        "miss_rate_measured": misses / (R * G * cfg["k"]),
-        "roofline": {"bound": "hbm", "kernel": SCAN_KERNEL if cfg["B"] <= 144 else "fathom_scan_topk (scan stage of the step)",
-                     "achieved": scan_bytes / (stages_ms["scan"] / 1e3) / 1e9, "peak": peak,
-                     "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": scan_bytes / (stages_ms["scan"] / 1e3) / 1e9 / peak,
-                     "traffic": TRAFFIC.get((args.workload, cfg["B"])),
-                     "algorithmic_bytes": scan_bytes, "ms": stages_ms["scan"],
-                     "bytes_moved": scan_bytes + algo["keys"] * (4 + 4 / 16) if cfg["B"] <= 144 else None},
-        "stages_ms": stages_ms,
-        "scan_only": {"kernel": "fathom_scan_lut (scores written to HBM)", "ms": scan_ms,
+        "layer_steps_per_s": head["layer_steps_per_s"],
+        "achieved_gbs": head["achieved_gbs"],
+        "step_frac_hbm": head["step_frac_hbm"],
+        "miss_rate_measured": head["miss_rate_measured"],
+        "roofline": head["roofline"],
+        "stages_ms": head["stages_ms"],
+        "scan_only": {"kernel": scan_kernel_name(B, False) + " (scores written to HBM)", "ms": scan_ms,
                       "achieved_gbs": scan_gbs, "frac": scan_gbs / peak},
         "e2e": {"value": keys_total / (e2e_ms / 1e3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk,
+        "clocks": head["clocks"],
     }
-    if rank == 0 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(cfg, data, rows=args.cpu_rows)
+    if "cpu_baseline" in head:
+        res["cpu_baseline"] = head["cpu_baseline"]
+    del step, hot, head
+    torch.cuda.empty_cache()
+
+    if not args.only_headline:
+        res["configs"] = other_configs(args, cfg, data, dist, ws, peak, bf16_peak, peak_kind)
+    del data
+    CLOCKS.stop()
+    res["clocks_all_legs"] = CLOCKS.window(-math.inf, math.inf)
+    return res
+
+
+def other_configs(args, cfg128, data128, dist, ws, peak, bf16_peak, peak_kind) -> dict:
+    """Every other workload of the scope, each timed like the headline."""
+    import kv_index_scan_b200 as kvs
+    dev = data128["K"].device
+    cpu_rows = 0 if args.no_cpu_baseline else 2
+    out = {}
+    for B in (68, 136, 512):
+        e = decode_entry("128k", cfg128, data128, B, args, dist, ws, peak, peak_kind, cpu_rows, 2.0)
+        out[f"128k-B{B}"] = _strip(e)
+        del e
+    data128.clear()
+    torch.cuda.empty_cache()
+
+    cfg1m = dict(WORKLOADS["qwen3-8b-1m"], name="qwen3-8b-1m")
+    d1 = setup_fathom(cfg1m, dev, seed=2 + (dist.get_rank() if dist else 0))
+    for B in (92, 136):
+        e = decode_entry("1m", cfg1m, d1, B, args, dist, ws, peak, peak_kind, cpu_rows, 2.0)
+        out[f"1m-B{B}"] = _strip(e)
+        del e
+    # the same layer with the index planes in mapped pinned host memory
+    hix = kvs.MappedHostIndex(d1["index"])
+    plane_bytes = int(algorithmic_bytes(cfg1m, 92)["scan"])
+    host_buf = torch.empty(plane_bytes, dtype=torch.uint8).pin_memory()
+    dev_buf = torch.empty(plane_bytes, dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        dev_buf.copy_(host_buf, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(5):
+        dev_buf.copy_(host_buf, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    link_gbs = 5 * plane_bytes / (e0.elapsed_time(e1) / 1e3) / 1e9
+    del host_buf, dev_buf
+    e = decode_entry("1m-host", cfg1m, d1, 92, args, dist, ws, peak, peak_kind, 0, 0.0,
+                     host_index=hix, link_peak=link_gbs)
+    e["pinned_copy_gbs"] = link_gbs
+    e["host_link_gbs"] = e["roofline"]["achieved"]
+    out["1m-host-B92"] = _strip(e)
+    del e, hix
+    d1.clear()
+    torch.cuda.empty_cache()
+
+    out["lightning-pair"] = lightning_entry(args, dist, peak, bf16_peak, peak_kind, cpu_rows > 0)
+    torch.cuda.empty_cache()
+    return out
+
+
+def lightning_entry(args, dist, peak, bf16_peak, peak_kind, with_cpu: bool) -> dict:
+    """The lightning layer pair: indexer (a2-L) + block top-k (a3) on layer 2j,
+    and the sparse attention of both layers of the group over that one
+    selection (a7), all KV heads of a request sharing it."""
+    import kv_index_scan_b200 as kvs
+    c = LIGHTNING
+    dev = torch.device("cuda", torch.cuda.current_device())
+    R, n, Hi, Dl, block, k, G, H = (c[x] for x in ("R", "n", "Hi", "Dl", "block", "k", "G", "H"))
+    kidx, qidx, w, nl = synth.lightning_inputs(R, n, Hi=Hi, Dl=Dl, seed=3, device=dev)
+    layers = []
+    for layer in range(2):
+        K, V, _ = synth.fathom_kv(R, G, 128, n, seed=40, layer=layer, device=dev)
+        q = synth.queries(R, G, H, 128, seed=40, layer=layer, device=dev, dtype=torch.bfloat16)
+        ix = kvs.build_fathom_index(K[:1, :1, :32], [32])  # not read: the selection is given
+        st = kvs.DecodeStep(ix, nl, n, H, 92, k, K, V, q_dtype=torch.bfloat16)
+        layers.append((q, st))
+    nb = (n + block - 1) // block
+    bs = torch.empty(R, nb, dtype=torch.float32, device=dev)
+    idx = torch.empty(R, 1, k, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def pair(ev=None):
+        if ev:
+            ev[0].record(stream)
+        kvs.index_scan_lightning(kidx, qidx, w, nl, block=block, scores=bs)
+        if ev:
+            ev[1].record(stream)
+        kvs.topk_select(bs, nl, k, block=block, idx=idx)
+        if ev:
+            ev[2].record(stream)
+        for j, (q, st) in enumerate(layers):
+            st(q, idx_in=idx, idx_shared=True)
+            if ev:
+                ev[3 + j].record(stream)
+
+    for _ in range(args.warmup):
+        pair()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    with Region() as reg:
+        for i in range(args.steps):
+            pair(evs[i])
+        torch.cuda.synchronize()
+    t = lambda a, b: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
+    scan_ms, topk_ms, a1_ms, a2_ms, pair_ms = t(0, 1), t(1, 2), t(2, 3), t(3, 4), t(0, 4)
+    kbytes = R * n * Dl
+    flops = 2.0 * R * n * Hi * Dl
+    rows = R * G * k * 2 * 128 * 2  # K and V rows of one layer
+    pair_bytes = kbytes + 2 * rows
+    scan_gbs = kbytes / (scan_ms / 1e3) / 1e9
+    res = {"workload": "minimax-lightning-32x80000", "requests": R, "tokens": n,
+           "index_heads": Hi, "block": block, "topk": k, "kv_heads": G, "q_heads_per_kv": H,
+           "ms_per_layer_pair": pair_ms, "layer_pairs_per_s": 1e3 / pair_ms,
+           "index_keys_per_s": R * n / (scan_ms / 1e3),
+           "stages_ms": {"indexer": scan_ms, "block_topk": topk_ms, "attention_layer0": a1_ms,
+                         "attention_layer1": a2_ms},
+           "pair_achieved_gbs": pair_bytes / (pair_ms / 1e3) / 1e9,
+           "pair_frac_hbm": pair_bytes / (pair_ms / 1e3) / 1e9 / peak,
+           "indexer_tflops": flops / (scan_ms / 1e3) / 1e12,
+           "indexer_frac_tensor": flops / (scan_ms / 1e3) / 1e12 / bf16_peak,
+           "roofline": {"bound": "hbm", "kernel": "lightning_scan (tcgen05 kind::f16)",
+                        "achieved": scan_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                        "frac": scan_gbs / peak, "traffic": None, "algorithmic_bytes": kbytes,
+                        "ms": scan_ms},
+           "clocks": reg.clocks()}
+    if with_cpu and (dist is None or dist.get_rank() == 0):
+        import oracle
+        cores = os.cpu_count() or 1
+        reps, t0 = 0, time.perf_counter()
+        sub_k = kidx[:1].cpu()
+        sub_q, sub_w = qidx[:1].cpu(), w[:1].cpu()
+        while True:
+            oracle.lightning_batch(sub_k, sub_q, sub_w, [n], block, k, nthreads=cores)
+            reps += 1
+            dt = time.perf_counter() - t0
+            if dt >= 2.0:
+                break
+        res["cpu_baseline"] = {"value": reps * n / dt, "unit": "index keys/s", "cores": cores,
+                               "kind": "oracle",
+                               "sample": f"the indexer and block top-k of 1 of {R} requests "
+                                         f"({n} tokens x {Hi} heads) x {reps} repetitions, fp64 "
+                                         f"C++ oracle, {dt:.1f} s"}
+    del layers
     return res
 
 
@@ -366,43 +645,9 @@ def step_needs_combine(cfg) -> bool:
     return kvs._lib.kvs_attn_workspace_size(cfg["R"], cfg["G"], cfg["H"], cfg["k"]) > 0
 
 
-def cpu_baseline(cfg, data, rows: int = 8, min_seconds: float = 10.0) -> dict:
-    """The CPU oracle, as it stands, on a bounded sample of the same workload:
-    `rows` (request, KV head) rows of the decode step, all host cores."""
-    import oracle
-    R, G, H, n, B, k = (cfg[x] for x in ("R", "G", "H", "n", "B", "k"))
-    rows = min(rows, R * G)
-    us = list(range(rows))
-    rr = [u // G for u in us]
-    gg = [u % G for u in us]
-    K = data["K"][rr, gg].unsqueeze(0).cpu()
-    V = data["V"][rr, gg].unsqueeze(0).cpu()
-    q = data["q"][rr, gg].unsqueeze(0).cpu()
-    nl = [data["nl"][0]]
-    sm = data["slot_map"][rr, gg].unsqueeze(0).cpu()
-    hK = data["hotK"][rr, gg].unsqueeze(0).cpu()
-    hV = data["hotV"][rr, gg].unsqueeze(0).cpu()
-    W = synth.plane_words(n)
-    planes, kmin, kstep, kvar = oracle.build_index_batch(K, nl, W)  # data prep, not timed
-    cores = os.cpu_count() or 1
-    reps, t0 = 0, time.perf_counter()
-    while True:  # repeat the bounded sample until ~10 s of CPU work
-        oracle.decode_batch(q, planes, kmin, kstep, kvar, nl, B, k, sm, hK, hV, K, V,
-                            1 / math.sqrt(128), nthreads=cores)
-        reps += 1
-        dt = time.perf_counter() - t0
-        if dt >= min_seconds or reps >= 5000:
-            break
-    return {"value": reps * rows * n / dt, "unit": "keys/s", "cores": cores, "kind": "oracle",
-            "sample": f"{rows} of {R * G} (request, KV head) rows of one decode step "
-                      f"({rows * n} keys) x {reps} repetitions, fp64 C++ oracle on {cores} "
-                      f"threads, {dt:.1f} s"}
-
-
 def run_reference(args, cfg, dist, rank, ws):
     """The CPU oracle timed as the reference arm, on the same workload's shape."""
     import oracle
-    dev = torch.device("cuda", torch.cuda.current_device()) if torch.cuda.is_available() else "cpu"
     R, G, H, n, B, k, S = (cfg[x] for x in ("R", "G", "H", "n", "B", "k", "S"))
     rows = min(args.cpu_rows, R * G)
     # a sample of rows of the same workload: (rows requests x 1 head) of length n
@@ -457,21 +702,22 @@ def _time_ms(fn, steps: int, warmup: int) -> float:
 
 
 def run_row(args) -> dict:
-    """Measurements of single rows of the path outside the default decode step
-    (one JSON line each; not the benchmark's headline line):
-      lightning -- the lightning indexer (a2-L) and its block top-k (a3, block
-                   64) at 32 requests x 80000 tokens x 64 index heads;
+    """Measurements of single rows of the path outside the decode step (one
+    JSON line each; not the benchmark's headline line):
+      lightning -- the lightning indexer (a2-L) alone and its block top-k (a3,
+                   block 64) at 32 requests x 80000 tokens x 64 index heads,
+                   two input sets in turn;
       host-scan -- the Fathom scan reading its planes from mapped pinned host
                    memory (a2-host) at the 1M layer (4 x 8 x 1048576, B = 92),
                    beside the same scan from HBM and a pinned host-to-device
                    copy of the same size (the link's copy rate)."""
     import kv_index_scan_b200 as kvs
     dev = torch.device("cuda")
-    peak, peak_kind = _peaks()
+    peak, bf16_peak, peak_kind = _peaks()
     steps, warmup = max(args.steps, 5), max(args.warmup, 3)
     if args.row == "lightning":
-        R, n, Hi, Dl, block, k = 32, 80000, 64, 128, 64, 2048
-        # two input sets in turn (each 328 MB of index keys, more than L2)
+        c = LIGHTNING
+        R, n, Hi, Dl, block, k = (c[x] for x in ("R", "n", "Hi", "Dl", "block", "k"))
         sets = [synth.lightning_inputs(R, n, Hi, Dl, seed=3 + j, device=dev) for j in range(2)]
         nb = (n + block - 1) // block
         bs = torch.empty(R, nb, dtype=torch.float32, device=dev)
@@ -504,7 +750,6 @@ def run_row(args) -> dict:
                            min(steps, 10), 2)
         host_vs_hbm = float((ref - scores).abs().max())
         plane_bytes = R * G * n * B / 8
-        # the link's copy rate for the same byte count, from pinned host memory
         host_buf = torch.empty(int(plane_bytes), dtype=torch.uint8).pin_memory()
         dev_buf = torch.empty(int(plane_bytes), dtype=torch.uint8, device=dev)
         copy_ms = _time_ms(lambda i: dev_buf.copy_(host_buf, non_blocking=True), 5, 2)
@@ -533,27 +778,29 @@ def main():
     ap.add_argument("--requests", type=int, default=None,
                     help="override the workload's request count (smaller profiling cases)")
     ap.add_argument("--only-step", action="store_true",
-                    help="time the decode steps only (no scan-alone, end-to-end or CPU legs); "
-                         "prints the step and stage times, for profiling runs")
+                    help="time the decode steps only (no scan-alone, end-to-end, CPU or other "
+                         "workloads); prints the step and stage times, for profiling runs")
+    ap.add_argument("--only-headline", action="store_true",
+                    help="measure the headline workload only (no other workloads)")
     ap.add_argument("--row", default=None, choices=["lightning", "host-scan"],
                     help="measure one row of the path outside the decode step (one JSON line)")
     args = ap.parse_args()
     if args.row is not None:
         print(json.dumps(run_row(args)), flush=True)
         return
-    cfg = dict(WORKLOADS[args.workload])
-    if args.B is not None:
-        cfg["B"] = args.B
-    if args.requests is not None:
-        cfg["R"] = args.requests
     if args.impl == "reference":
+        cfg = dict(WORKLOADS[args.workload])
+        if args.B is not None:
+            cfg["B"] = args.B
+        if args.requests is not None:
+            cfg["R"] = args.requests
         # the CPU oracle: rank 0 alone runs it; other ranks exit without work
         if int(os.environ.get("RANK", "0")) == 0:
             ws = int(os.environ.get("WORLD_SIZE", "1"))
             print(json.dumps(run_reference(args, cfg, None, 0, ws)), flush=True)
         return
     dist, rank, ws = _dist()
-    res = run_ours(args, cfg, dist, rank, ws)
+    res = run_ours(args, dist, rank, ws)
     if rank == 0 and res is not None:
         print(json.dumps(res), flush=True)
     if dist:

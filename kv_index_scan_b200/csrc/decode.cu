@@ -8,6 +8,8 @@
 // group sharing of "MiniMax-M3: share the sparse index top-k across layers and
 // reuse the decode top-k buffer" (description), where the group's first layer
 // selects and the others reuse the selection.
+#include <algorithm>
+
 #include "internal.cuh"
 #include "scan_core.cuh"
 
@@ -42,8 +44,11 @@ size_t decode_ws_bytes(int R, int G, int H, int n_max, int k, int B) {
   c.take<int32_t>(static_cast<size_t>(R) * G * k);  // slots when the caller passes none
   c.take<unsigned char>(attn_ws_bytes(R * G, H, k));
   const size_t unfused = static_cast<size_t>(R) * G * n_max * sizeof(float);  // scores
+  // the larger of the HBM and the host-mapped layouts (the index's residence
+  // is not known here)
   const size_t fused = fused_topk_supported(n_max, k, B)
-                           ? fused_ws_bytes(R * G, n_max, k, B) : 0;
+                           ? std::max(fused_ws_bytes(R * G, n_max, k, B),
+                                      fused_ws_bytes(R * G, n_max, k, B, true)) : 0;
   c.take<unsigned char>(unfused > fused ? unfused : fused);
   return c.used;
 }
@@ -72,9 +77,11 @@ kvs_status decode_step_run(const kvs_decode_args* a, void* ws, int32_t* dev_stat
                           a->plan->C, s);
     if (st != KVS_OK) return st;
     mark(1);
-    if (!a->ix->host_mapped && fused_topk_supported(a->n_max, a->k, B)) {
-      // scan with on-chip top-k candidates, then the per-row merge (which also
-      // writes the slots and misses)
+    if (fused_topk_supported(a->n_max, a->k, B)) {
+      // plans of <= 144 planes or an index in mapped host memory: the scan
+      // writes scores and 16-key maxima, then the per-row top-k over them;
+      // longer plans: the scan keeps top-k candidates on chip, then the
+      // per-row merge (both write the slots and misses)
       ScanParams p{};
       p.planes = a->ix->planes;
       p.W = a->ix->W;
@@ -90,7 +97,7 @@ kvs_status decode_step_run(const kvs_decode_args* a, void* ws, int32_t* dev_stat
       p.dev_status = dev_status;
       p.k = a->k;
       st = fathom_scan_topk_launch(p, rest, a->slot_map, a->idx, slots, a->misses, s,
-                                   ev ? ev[2] : nullptr);
+                                   ev ? ev[2] : nullptr, a->ix->host_mapped != 0);
       if (st != KVS_OK) return st;
       have_slots = true;
     } else {

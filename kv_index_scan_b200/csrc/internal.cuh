@@ -34,14 +34,14 @@ kvs_status plan_bits_launch(const float* q, int H, const float* kmin, const floa
 kvs_status fathom_scan_simple_launch(const uint32_t* planes, int W, int R, int G,
                                      const uint16_t* plane_idx, const float* plane_w,
                                      const float* C, int B, const int32_t* n, int n_max,
-                                     float* scores, cudaStream_t s);
+                                     float* scores, cudaStream_t s, float* gmax = nullptr);
 struct ScanParams;
 kvs_status fathom_scan_lut_launch(const ScanParams& p, cudaStream_t s);
 bool fused_topk_supported(int n_max, int k, int B);
-size_t fused_ws_bytes(int RG, int n_max, int k, int B);
+size_t fused_ws_bytes(int RG, int n_max, int k, int B, bool host_mapped = false);
 kvs_status fathom_scan_topk_launch(ScanParams p, void* ws, const int32_t* slot_map, int32_t* idx,
                                    int32_t* slots, int32_t* misses, cudaStream_t s,
-                                   cudaEvent_t after_scan = nullptr);
+                                   cudaEvent_t after_scan = nullptr, bool host_mapped = false);
 kvs_status fathom_scan_dispatch(const kvs_fathom_index* ix, const kvs_plan* plan,
                                 const int32_t* n, int n_max, float* scores, int32_t* dev_status,
                                 cudaStream_t s);

@@ -1170,8 +1170,8 @@ bool fused_topk_supported(int n_max, int k, int B) {
          n_max <= (1 << kIdxBits);
 }
 
-size_t fused_ws_bytes(int RG, int n_max, int k, int B) {
-  if (B <= kPMaxB) {
+size_t fused_ws_bytes(int RG, int n_max, int k, int B, bool host_mapped) {
+  if (B <= kPMaxB || host_mapped) {
     WsCarver c(nullptr);
     c.take<float>(static_cast<size_t>(RG) * n_max);
     c.take<float>(static_cast<size_t>(RG) * ((n_max + kPKeys - 1) / kPKeys));
@@ -1196,8 +1196,8 @@ size_t fused_ws_bytes(int RG, int n_max, int k, int B) {
 
 kvs_status fathom_scan_topk_launch(ScanParams p, void* ws, const int32_t* slot_map, int32_t* idx,
                                    int32_t* slots, int32_t* misses, cudaStream_t s,
-                                   cudaEvent_t after_scan) {
-  if (p.B <= kPMaxB) {
+                                   cudaEvent_t after_scan, bool host_mapped) {
+  if (p.B <= kPMaxB || host_mapped) {
     // scores and 16-key group maxima from the byte-indexed scan, then the
     // per-row top-k over them
     WsCarver c(ws);
@@ -1205,7 +1205,11 @@ kvs_status fathom_scan_topk_launch(ScanParams p, void* ws, const int32_t* slot_m
     q.scores = c.take<float>(static_cast<size_t>(p.RG) * p.n_max);
     q.gmax = c.take<float>(static_cast<size_t>(p.RG) * ((p.n_max + kPKeys - 1) / kPKeys));
     uint32_t* bitmap = c.take<uint32_t>(static_cast<size_t>(p.RG) * bitmap_words(p.n_max));
-    kvs_status st = fathom_scan_lut_launch(q, s);
+    // the index in mapped host memory: the plain scan, reading over the host link
+    kvs_status st = host_mapped
+                        ? fathom_scan_simple_launch(p.planes, p.W, p.RG / p.Gheads, p.Gheads, p.plane_idx,
+                                                    p.plane_w, p.C, p.B, p.n, p.n_max, q.scores, s, q.gmax)
+                        : fathom_scan_lut_launch(q, s);
     if (st != KVS_OK) return st;
     if (after_scan) cudaEventRecord(after_scan, s);
     cudaFuncSetAttribute(topk_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
