@@ -18,6 +18,10 @@ workload, each timed with the same --steps/--warmup and each with its own
 roofline (algorithmic bytes of its dominant kernel / that kernel's CUDA-event
 time / the measured peak) and a short CPU-oracle sample:
   128k-B68, 128k-B136, 128k-B512  the 128K layer at the other budgets;
+  128k-hosttier-miss20, -miss40   the 128K step with the full K/V store in
+                                  mapped pinned host memory: the missing
+                                  selected rows (20% / 40%) cross the host link
+                                  each step; against the all-in-HBM step;
   1m-B92, 1m-B136                 the 1M layer (4 x 8 x 1048576), index in HBM;
   1m-host-B92                     the 1M layer with the index planes in mapped
                                   pinned host memory, read by the scan over
@@ -26,7 +30,17 @@ time / the measured peak) and a short CPU-oracle sample:
   lightning-pair                  32 requests x 80000 tokens: lightning
                                   indexer (64 heads, tcgen05), block top-k,
                                   and sparse attention for both layers of a
-                                  group reusing one selection.
+                                  group reusing one selection;
+  selection-quality               a diagnostic: top-k recall against the exact
+                                  bf16-K top-k and attention error against
+                                  dense attention, for the Fathom allocation
+                                  at 68/92/136 bits and a SparQ-like scan of
+                                  the B/4 largest-|qbar| channels at equal bits;
+  sweep-36-layers                 ragged batches of 1 .. 256 requests (lengths
+                                  log-uniform in [16K, 128K]) over 36 layers:
+                                  each batch's footprint against 180 GB, and for
+                                  the batches that fit, one layer's decode step
+                                  timed (the 36 layers have the same shape).
 --only-headline skips them.
 
 --impl reference times the CPU oracle (the only reference this method has) on
@@ -60,6 +74,9 @@ WORKLOADS = {
     "tiny": dict(R=1, G=1, H=4, n=4096, B=92, k=256, S=512, miss=0.2),
 }
 LIGHTNING = dict(R=32, n=80000, Hi=64, Dl=128, block=64, k=2048, G=8, H=4)
+# the concurrency sweep: ragged batches over 36 layers, capped by 180 GB of HBM
+SWEEP = dict(layers=36, batches=(1, 2, 4, 8, 16, 32, 64, 128, 256), G=8, H=4, B=92, k=2048, S=4096,
+             lo=16384, hi=131072, cap_gb=180.0, miss=0.2, seed=4)
 METRIC = "index-scan keys/s + sparse decode layer-steps/s; achieved GB/s vs HBM peak"
 
 # DRAM bytes (read + write) of one launch of the scan kernel, from ncu
@@ -515,6 +532,11 @@ def other_configs(args, cfg128, data128, dist, ws, peak, bf16_peak, peak_kind) -
         e = decode_entry("128k", cfg128, data128, B, args, dist, ws, peak, peak_kind, cpu_rows, 2.0)
         out[f"128k-B{B}"] = _strip(e)
         del e
+    hostK, hostV = kvs.MappedHostStore(data128["K"]), kvs.MappedHostStore(data128["V"])
+    for miss in (0.2, 0.4):
+        out[f"128k-hosttier-miss{round(100 * miss)}"] = hosttier_entry(cfg128, data128, miss, hostK, hostV,
+                                                                       args, dist)
+    del hostK, hostV
     data128.clear()
     torch.cuda.empty_cache()
 
@@ -551,6 +573,211 @@ def other_configs(args, cfg128, data128, dist, ws, peak, bf16_peak, peak_kind) -
 
     out["lightning-pair"] = lightning_entry(args, dist, peak, bf16_peak, peak_kind, cpu_rows > 0)
     torch.cuda.empty_cache()
+    out["sweep-36-layers"] = sweep_entry(args, dist, ws, peak, peak_kind, cpu_rows > 0)
+    torch.cuda.empty_cache()
+    out["selection-quality"] = quality_entry()
+    torch.cuda.empty_cache()
+    out["throughput-model"] = model_entry(out["sweep-36-layers"])
+    return out
+
+
+def model_entry(sweep: dict, hbm_budget: float = 150e9, miss: float = 0.2) -> dict:
+    """The offloaded system's throughput and capacity model
+    (kv_index_scan_b200.capacity) fed with the sweep's measured decode-step
+    times: compute = 36 x the measured layer step of each batch (misses read
+    from HBM, so no link time in it), plus the fetch of the missing selected
+    entries over each link the page models; batches above a configuration's
+    capacity (hot buffers + K-index in hbm_budget of HBM, the full KV in the
+    link's external memory) get no figure."""
+    from kv_index_scan_b200 import capacity as cm
+    fp = cm.qwen3_8b_like(layers=SWEEP["layers"])
+    rows = []
+    for e in sweep["batches"]:
+        if e.get("ms_per_layer_step") is None:
+            continue
+        b, n = e["batch"], int(e["mean_length"])
+        tc = SWEEP["layers"] * e["ms_per_layer_step"] / 1e3
+        links = {}
+        for name, link in cm.LINKS.items():
+            bmax = cm.batch_max(fp, n, hbm_budget, link["capacity"])
+            links[name] = {"batch_max": bmax,
+                           "tokens_per_s": cm.tokens_per_s(tc, fp, b, SWEEP["k"], miss, link["bandwidth"])
+                           if b <= bmax else None}
+        rows.append({"batch": b, "mean_length": n, "t_compute_ms": tc * 1e3, "ideal_tokens_per_s": b / tc,
+                     "links": links})
+    return {"model": "T_step = T_compute + batch * layers * k * miss * entry bytes / link bandwidth; "
+                     "batch <= min(HBM budget / (hot + index), external capacity / full KV)",
+            "layers": SWEEP["layers"], "hbm_budget_gb": hbm_budget / 1e9, "miss_rate": miss,
+            "links": {k: {"gbs": v["bandwidth"] / 1e9, "capacity_tb": v["capacity"] / 1e12}
+                      for k, v in cm.LINKS.items()},
+            "rows": rows}
+
+
+def sparq_channels(qbar: torch.Tensor, r: int) -> torch.Tensor:
+    """The r channels with the largest |qbar_c| per row, ties to the lower
+    channel: [..., D] -> [..., r] (ascending)."""
+    order = torch.sort(qbar.abs(), dim=-1, descending=True, stable=True).indices
+    return torch.sort(order[..., :r], dim=-1).values
+
+
+def quality_entry(R: int = 4, G: int = 8, H: int = 4, n: int = 131072, k: int = 2048,
+                  budgets=(68, 92, 136), seed: int = 5) -> dict:
+    """The selection-quality diagnostic of the Fathom abstract's comparison
+    (bytes read against attention error and agreement with the exact top-k),
+    on synthetic data: for each budget B, the Fathom allocation (decode_step)
+    and a SparQ-like scan at the same B bits per key -- all 4 planes of the
+    B/4 channels of largest |qbar_c| -- through the same scan and top-k
+    kernels. Recall = |selection & exact top-k| / k, where the exact top-k is
+    that of qbar . K over the bf16 keys; attention error = relative L2 error
+    of the attention output against the output over the exact top-k (the
+    target a selection approximates). Against dense attention over all n keys
+    every selection's error is large on these synthetic keys (the attention
+    mass is spread over all of them), so that figure is reported beside it."""
+    import kv_index_scan_b200 as kvs
+    dev = torch.device("cuda", torch.cuda.current_device())
+    K, V, nl = synth.fathom_kv(R, G, 128, n, seed=seed, device=dev)
+    q = synth.queries(R, G, H, 128, seed=seed, device=dev)
+    ix = kvs.build_fathom_index(K, nl)
+    qbar = ((q[:, :, 0] + q[:, :, 1]) + q[:, :, 2]) + q[:, :, 3]  # [R][G][D]
+    exact = torch.einsum("rgd,rgnd->rgn", qbar, K.float())
+    o_star = torch.topk(exact, k, dim=2).indices
+    scale = 1 / math.sqrt(128)
+    logits = torch.einsum("rghd,rgnd->rghn", q, K.float()) * scale
+    dense = torch.einsum("rghn,rgnd->rghd", torch.softmax(logits, dim=-1), V.float())
+    attn = kvs.DecodeStep(ix, nl, n, H, 92, k, K, V)  # attention over a given selection
+
+    def recall(sel):
+        hits = torch.zeros(R, G, device=dev)
+        for r in range(R):
+            for g in range(G):
+                hits[r, g] = torch.isin(sel[r, g], o_star[r, g]).sum()
+        return float(hits.mean() / k)
+
+    def attn_out(sel):
+        return attn(q, idx_in=sel.to(torch.int32).contiguous()).clone()
+
+    def rel(out, ref):
+        return float(((out - ref).norm(dim=-1) / ref.norm(dim=-1)).mean())
+
+    exact_out = attn_out(torch.sort(o_star, dim=2).values)
+    res = {"requests": R, "kv_heads": G, "context": n, "topk": k,
+           "exact_topk_error_vs_dense": rel(exact_out, dense), "budgets": []}
+    for B in budgets:
+        step = kvs.DecodeStep(ix, nl, n, H, B, k, K, V)
+        step(q)
+        fathom_sel = step.idx.clone()
+        # the SparQ-like plan: all 4 planes of the B/4 largest-|qbar| channels
+        r = B // 4
+        ch = sparq_channels(qbar, r)  # [R][G][r]
+        pidx = (4 * ch.unsqueeze(-1) + torch.arange(4, device=dev)).reshape(R, G, 4 * r)
+        kst = torch.gather(ix.kstep, 2, ch)
+        kmn = torch.gather(ix.kmin, 2, ch)
+        qc = torch.gather(qbar, 2, ch)
+        pw = (qc * kst).unsqueeze(-1) * torch.tensor([8.0, 4.0, 2.0, 1.0], device=dev)
+        plan = kvs.Plan(R, G, 128, 4 * r, dev)
+        plan.plane_idx.copy_(pidx.to(torch.int16))
+        plan.plane_w.copy_(pw.reshape(R, G, 4 * r))
+        plan.C.copy_((qc * kmn).sum(-1))
+        sc = kvs.index_scan_fathom(ix, plan, nl, n)
+        sparq_sel = kvs.topk_select(sc, nl, k)
+        fo, so = attn_out(fathom_sel), attn_out(sparq_sel)
+        res["budgets"].append({"bits_per_key": B, "bytes_per_key": B / 8,
+                               "fathom_recall": recall(fathom_sel), "sparq_like_recall": recall(sparq_sel),
+                               "fathom_attention_error": rel(fo, exact_out),
+                               "sparq_like_attention_error": rel(so, exact_out),
+                               "fathom_error_vs_dense": rel(fo, dense),
+                               "sparq_like_error_vs_dense": rel(so, dense),
+                               "sparq_like_channels": r})
+    torch.cuda.synchronize()
+    return res
+
+
+def hosttier_entry(cfg, data, miss, hostK, hostV, args, dist) -> dict:
+    """The decode step with its full K/V store in the host tier (mapped
+    pinned host memory): each step fetches the missing selected rows over the
+    host link into HBM, then attends. Timed beside the same step with the
+    store in HBM; the fetch rate is the miss bytes over the extra time."""
+    import kv_index_scan_b200 as kvs
+    c = dict(cfg, miss=miss)
+    step_hbm, hot = decode_step_for(c, data, cfg["B"])
+    ms_hbm, _, _ = time_decode_steps(step_hbm, data["q"], args.steps, args.warmup, dist)
+    step = kvs.DecodeStep(data["index"], data["nl"], cfg["n"], cfg["H"], cfg["B"], cfg["k"], hostK, hostV,
+                          hot["slot_map"], hot["hotK"], hot["hotV"])
+    ms, stages, reg = time_decode_steps(step, data["q"], args.steps, args.warmup, dist)
+    ms_hbm, ms = _max_over_ranks(dist, ms_hbm), _max_over_ranks(dist, ms)
+    torch.cuda.synchronize()
+    same = bool(torch.equal(step.out, step_hbm.out) and torch.equal(step.idx, step_hbm.idx))
+    misses = int(step.misses.sum().item())
+    miss_bytes = misses * 2 * 128 * 2
+    extra = max(ms - ms_hbm, 1e-6)
+    return {"workload": cfg["name"], "full_store": "mapped pinned host memory", "miss_rate": miss,
+            "miss_rate_measured": misses / (cfg["R"] * cfg["G"] * cfg["k"]),
+            "ms_per_step": ms, "ms_per_step_all_in_hbm": ms_hbm, "layer_steps_per_s": 1e3 / ms,
+            "miss_bytes_per_step": miss_bytes, "fetch_gbs": miss_bytes / (extra / 1e3) / 1e9,
+            "stages_ms": stages, "outputs_equal_hbm_step": same, "clocks": reg.clocks()}
+
+
+def sweep_footprint(nl, c=SWEEP) -> dict:
+    """HBM bytes of a batch with lengths nl over c['layers'] layers: per
+    request and layer the index planes (4 planes of D channels, W words each),
+    the slot map and the hot K/V buffers; per request one full K/V store that
+    the layers share (it only serves the misses: a synthetic shortcut)."""
+    G, S = c["G"], c["S"]
+    per_layer = sum(G * 128 * 4 * synth.plane_words(n) * 4 + G * n * 4 + 2 * G * S * 128 * 2 for n in nl)
+    full = sum(2 * G * n * 128 * 2 for n in nl)
+    total = c["layers"] * per_layer + full
+    return {"bytes": total, "gb": total / 1e9, "over_capacity": total / 1e9 > c["cap_gb"]}
+
+
+def sweep_entry(args, dist, ws, peak, peak_kind, with_cpu: bool) -> dict:
+    """The concurrency sweep of the fused decode step (a6) over ragged
+    batches: layer-steps/s, 36-layer token steps/s and GB/s per batch size."""
+    import kv_index_scan_b200 as kvs
+    c = SWEEP
+    dev = torch.device("cuda", torch.cuda.current_device())
+    rank = dist.get_rank() if dist else 0
+    out = {"layers": c["layers"], "cap_gb": c["cap_gb"], "bits_per_key": c["B"], "topk": c["k"],
+           "hot_slots": c["S"], "miss_rate": c["miss"], "lengths": "floor(exp(U(ln 16384, ln 131072)))",
+           "timed": "one layer's fused decode step over the whole batch; the 36 layers have the same shape",
+           "batches": []}
+    for b in c["batches"]:
+        nl = synth.ragged_lengths(b, seed=c["seed"] * 1000 + b + 7919 * rank)
+        fp = sweep_footprint(nl)
+        e = {"batch": b, "mean_length": sum(nl) / b, "footprint_gb": fp["gb"],
+             "over_capacity": fp["over_capacity"]}
+        # every rank takes the same collective steps, fit or not
+        if fp["over_capacity"]:
+            out["batches"].append(e)
+            continue
+        n_max = max(nl)
+        K, V, _ = synth.fathom_kv(b, c["G"], 128, nl, n_max=n_max, seed=c["seed"] + 10 * rank, device=dev)
+        q = synth.queries(b, c["G"], c["H"], 128, seed=c["seed"] + 10 * rank, device=dev)
+        index = kvs.build_fathom_index(K, nl)
+        cfg = dict(R=b, G=c["G"], H=c["H"], n=n_max, B=c["B"], k=c["k"], S=c["S"], miss=c["miss"])
+        step, _ = decode_step_for(cfg, dict(K=K, V=V, q=q, index=index, nl=nl, seed=c["seed"]), c["B"])
+        ms, stages, reg = time_decode_steps(step, q, args.steps, args.warmup, dist)
+        ms = _max_over_ranks(dist, ms)
+        keys = c["G"] * sum(nl)
+        scan_bytes = keys * c["B"] / 8
+        rows = b * c["G"] * c["k"] * (2 * 128 * 2 + 32)
+        e.update({"ms_per_layer_step": ms, "layer_steps_per_s": 1e3 / ms,
+                  "token_steps_per_s": 1e3 / (ms * c["layers"]),
+                  "keys_per_s": keys * ws / (ms / 1e3),
+                  "achieved_gbs": (scan_bytes + rows) * ws / (ms / 1e3) / 1e9,
+                  "frac_hbm": (scan_bytes + rows) / (ms / 1e3) / 1e9 / peak,
+                  "stages_ms": stages, "clocks": reg.clocks()})
+        out["batches"].append(e)
+        if with_cpu and rank == 0 and b == 1:
+            data = dict(K=K, V=V, q=q, nl=nl, seed=c["seed"])
+            hot = {"slot_map": step.slot_map, "hotK": step.hotK, "hotV": step.hotV}
+            cb = oracle_sample(cfg, data, c["B"], hot, rows=2, min_seconds=2.0)
+            cb["sample"] += " (batch 1, one layer)"
+            out["cpu_baseline"] = cb
+        del K, V, q, index, step
+        torch.cuda.empty_cache()
+    fits = [e["batch"] for e in out["batches"] if not e["over_capacity"]]
+    out["largest_batch_that_fits"] = max(fits) if fits else 0
+    out["peak_kind"] = peak_kind
     return out
 
 
@@ -702,6 +929,12 @@ def _time_ms(fn, steps: int, warmup: int) -> float:
 
 
 def run_row(args) -> dict:
+    if args.row == "quality":
+        return quality_entry()
+    return _run_row(args)
+
+
+def _run_row(args) -> dict:
     """Measurements of single rows of the path outside the decode step (one
     JSON line each; not the benchmark's headline line):
       lightning -- the lightning indexer (a2-L) alone and its block top-k (a3,
@@ -782,7 +1015,7 @@ def main():
                          "workloads); prints the step and stage times, for profiling runs")
     ap.add_argument("--only-headline", action="store_true",
                     help="measure the headline workload only (no other workloads)")
-    ap.add_argument("--row", default=None, choices=["lightning", "host-scan"],
+    ap.add_argument("--row", default=None, choices=["lightning", "host-scan", "quality"],
                     help="measure one row of the path outside the decode step (one JSON line)")
     args = ap.parse_args()
     if args.row is not None:

@@ -313,6 +313,13 @@ KVS_API kvs_status sparse_decode_attn_noalloc(const void* q, int32_t q_dtype, co
  *   shared by all G heads (the lightning indexer's block selection);
  *   otherwise [R][G][k].
  * slot_map == NULL: rows come straight from fullK/fullV (no hot buffer).
+ * fullK/fullV may be page-locked host memory mapped into the device's address
+ *   space (the full store in the host tier, [XMSPARSE] Figure 1): the step
+ *   then reads the missing selected rows over the host link into a staging
+ *   area of the workspace and the attention reads every row from HBM (hits
+ *   from the hot buffer, misses from the staging); the results are those of
+ *   the all-in-HBM step, bit for bit. The workspace must then be
+ *   kvs_decode_step_workspace_size_host() bytes (KVS_EWORKSPACE otherwise).
  *
  * Outputs: out f32 [R][G][H][D]; lse (nullable) [R][G][H]; idx (written only
  * when idx_in == NULL) [R][G][k]; slots (nullable) [R][G][k]; misses
@@ -345,6 +352,58 @@ KVS_API kvs_status decode_step(const kvs_decode_args* a, void* ws, size_t ws_byt
                        void* stream);
 KVS_API size_t kvs_decode_step_workspace_size(int32_t R, int32_t G, int32_t H, int32_t n_max, int32_t k,
                                       int32_t B);
+/* Workspace of decode_step when fullK/fullV are in host memory: the above
+ * plus two [R][G][k][D] bf16 staging buffers for the fetched misses. */
+KVS_API size_t kvs_decode_step_workspace_size_host(int32_t R, int32_t G, int32_t H, int32_t n_max,
+                                                   int32_t k, int32_t B);
+
+/* ---------------------------------------------------------------------------
+ * kvs_append_token -- the per-step write-back after a decode step: the token
+ * just generated joins every (request, KV head) row [XMSPARSE, the request
+ * lifecycle list: the generated KV is written back at each step; FATHOM: the
+ * 4-bit bit-plane K copy the scan reads].
+ *
+ * For each request r with i = n[r] < n_max: channel c of KV head g gets the
+ * code u = clamp(floor((k - m_c) / s_c + 1/2), 0, 15), computed in fp64 from
+ * the bf16 key Knew[r][g][c] with the row's stored kmin/kstep (s_c = 0 -> 0):
+ * the quantiser of kvs_build_fathom_index, not re-fitted (kmin, kstep and
+ * kvar are left as they are, so a key outside the row's range takes the end
+ * code). The four plane bits of key i are set to u's bits (plane 0 = MSB),
+ * fullK/fullV[r][g][i] receive Knew/Vnew[r][g], and n[r] grows by one.
+ * Slot map and hot buffer (all nullable): without hot_slot, slot_map[r][g][i]
+ * (if given) is set to -1 (a miss until a hot-buffer policy brings it in);
+ * with hot_slot [R][G], a slot s = hot_slot[r][g] >= 0 receives the new rows
+ * in hotK/hotV[r][g][s], the token it held before (hot_tok[r][g][s], -1 when
+ * empty) leaves the slot map (slot_map = -1), and hot_tok[r][g][s] = i,
+ * slot_map[r][g][i] = s. A request already at n[r] == n_max is left
+ * unchanged and KVS_EBOUNDS is written to dev_status.
+ *   Knew, Vnew bf16 [R][G][D]; n device int32 [R] (read and advanced);
+ *   planes u32 [R][G][D][4][W] (written); kmin, kstep f32 [R][G][D];
+ *   fullK, fullV bf16 [R][G][n_max][D]; slot_map i32 [R][G][n_max];
+ *   hot_slot i32 [R][G]; hot_tok i32 [R][G][S]; hotK, hotV bf16 [R][G][S][D].
+ * D = 128, G <= 8. The pages define no such call signature; it is the
+ * write-back step of their request lifecycle. */
+KVS_API kvs_status kvs_append_token(const uint16_t* Knew, const uint16_t* Vnew, int32_t* n, int32_t R,
+                                    int32_t G, int32_t D, int32_t n_max, uint32_t* planes, int32_t W,
+                                    const float* kmin, const float* kstep, uint16_t* fullK,
+                                    uint16_t* fullV, int32_t* slot_map, const int32_t* hot_slot,
+                                    int32_t* hot_tok, uint16_t* hotK, uint16_t* hotV, int32_t S,
+                                    int32_t* dev_status, void* stream);
+
+/* kvs_selftest_scan_timeout -- a check of the bounded waits, without a GPU
+ * fault: runs the HBM Fathom scan of index_scan (index in HBM, a plan of
+ * 1..144 planes) with one producer warp of every block withholding its
+ * arrival on its first chunk and every wait bounded by wait_cycles
+ * (1e3 .. 2e9 SM cycles; the library's waits are otherwise bounded by 2e9,
+ * about one second). The consumers' wait for that chunk runs out: they write
+ * KVS_ETIMEOUT to dev_status (required here), stop waiting, the producers
+ * see the block's abort flag, and every block returns with no copy in
+ * flight, leaving the context usable. The scores it writes are not
+ * meaningful. For tests of the failure path only; the pages define no such
+ * call. */
+KVS_API kvs_status kvs_selftest_scan_timeout(const kvs_fathom_index* ix, const kvs_plan* plan,
+                                             const int32_t* n, int32_t n_max, float* scores,
+                                             int64_t wait_cycles, int32_t* dev_status, void* stream);
 
 /* decode_step_timed -- decode_step that also records caller-created CUDA
  * events (cudaEvent_t handles, passed as void*) on `stream` at the boundaries

@@ -90,8 +90,16 @@ def _declare():
     L.decode_step.restype = I32
     L.kvs_decode_step_workspace_size.argtypes = [I32, I32, I32, I32, I32, I32]
     L.kvs_decode_step_workspace_size.restype = SZ
+    L.kvs_decode_step_workspace_size_host.argtypes = [I32, I32, I32, I32, I32, I32]
+    L.kvs_decode_step_workspace_size_host.restype = SZ
     L.decode_step_timed.argtypes = [ctypes.POINTER(DecodeArgsC), P, SZ, P, P, ctypes.POINTER(P), I32]
     L.decode_step_timed.restype = I32
+    L.kvs_append_token.argtypes = [P, P, P, I32, I32, I32, I32, P, I32, P, P, P, P, P, P, P, P, P, I32,
+                                   P, P]
+    L.kvs_append_token.restype = I32
+    L.kvs_selftest_scan_timeout.argtypes = [ctypes.POINTER(FathomIndexC), ctypes.POINTER(PlanC), P, I32,
+                                            P, I64, P, P]
+    L.kvs_selftest_scan_timeout.restype = I32
 
 
 _declare()
@@ -118,6 +126,8 @@ def _ptr(t) -> int | None:
         return None
     if isinstance(t, int):
         return t
+    if isinstance(t, MappedHostStore):
+        return t.ptr
     return t.data_ptr()
 
 
@@ -128,7 +138,7 @@ def _stream(stream=None) -> int | None:
 
 
 def _u16(t):
-    return t.view(torch.int16) if t is not None and t.dtype == torch.bfloat16 else t
+    return t.view(torch.int16) if isinstance(t, torch.Tensor) and t.dtype == torch.bfloat16 else t
 
 
 def plane_words(n_max: int) -> int:
@@ -181,6 +191,38 @@ class MappedHostIndex(FathomIndex):
         super().__init__(index.planes, index.kmin, index.kstep, index.kvar, planes_ptr=int(dptr),
                          host_mapped=True)
         self.nbytes = nbytes
+
+    def __del__(self):
+        try:
+            self._rt.cudaFreeHost(self._hptr)
+        except Exception:
+            pass
+
+
+class MappedHostStore:
+    """A full K or V store in mapped pinned host memory (cudaHostAlloc with
+    cudaHostAllocMapped): the host tier of the pages' system. `ptr` is its
+    device alias, which decode_step reads over the host link (only the missing
+    selected rows). Built from a bf16 device tensor [R][G][n_max][D]; the host
+    buffer is freed when this object is."""
+
+    def __init__(self, t: torch.Tensor):
+        from cuda.bindings import runtime as rt
+        self._rt = rt
+        self.shape = tuple(t.shape)
+        self.nbytes = t.numel() * t.element_size()
+        err, hptr = rt.cudaHostAlloc(self.nbytes, rt.cudaHostAllocMapped | rt.cudaHostAllocPortable)
+        if err != rt.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"cudaHostAlloc: {err}")
+        self._hptr = hptr
+        err, dptr = rt.cudaHostGetDevicePointer(hptr, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"cudaHostGetDevicePointer: {err}")
+        torch.cuda.synchronize()
+        err, = rt.cudaMemcpy(hptr, t.data_ptr(), self.nbytes, rt.cudaMemcpyKind.cudaMemcpyDeviceToHost)
+        if err != rt.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"cudaMemcpy: {err}")
+        self.ptr = int(dptr)
 
     def __del__(self):
         try:
@@ -367,6 +409,40 @@ def sparse_decode_attn_noalloc(q, K, V, out, lse=None, k_eff=None, scale: float 
     return out, lse
 
 
+def append_token(index: FathomIndex, Knew, Vnew, n: torch.Tensor, fullK, fullV, slot_map=None,
+                 hot_slot=None, hot_tok=None, hotK=None, hotV=None, stream=None, dev_status=None):
+    """Per-step write-back (kvs_append_token): the new token Knew/Vnew bf16
+    [R][G][D] of every request joins its rows at position n[r] -- its 4-bit
+    codes (the index's own quantiser) into the planes, its K/V rows into the
+    full store, optionally a hot slot (hot_slot int32 [R][G], with hot_tok
+    int32 [R][G][S] the token each slot holds) -- and n (device int32 [R]) is
+    advanced in place."""
+    R, G, D = Knew.shape
+    n_max = fullK.shape[2]
+    if n.dtype != torch.int32 or not n.is_contiguous() or n.device != Knew.device:
+        raise ValueError("n must be a contiguous device int32 tensor on Knew's device")
+    S = hotK.shape[2] if hotK is not None else 0
+    st = _lib.kvs_append_token(_ptr(_u16(Knew)), _ptr(_u16(Vnew)), _ptr(n), R, G, D, n_max,
+                               _ptr(index.planes), index.W, _ptr(index.kmin), _ptr(index.kstep),
+                               _ptr(_u16(fullK)), _ptr(_u16(fullV)), _ptr(slot_map), _ptr(hot_slot),
+                               _ptr(hot_tok), _ptr(_u16(hotK)), _ptr(_u16(hotV)), S,
+                               _ptr(dev_status), _stream(stream))
+    _check(st, "kvs_append_token")
+
+
+def selftest_scan_timeout(index: FathomIndex, plan: Plan, n, n_max: int, wait_cycles: int,
+                          dev_status: torch.Tensor, stream=None):
+    """kvs_selftest_scan_timeout: the HBM scan with a withheld producer
+    arrival, so that its bounded waits run out; dev_status (device int32)
+    receives KVS_ETIMEOUT. For tests of the failure path."""
+    nt = _n_tensor(n, index.R, index.kmin.device)
+    scores = torch.empty(index.R, index.G, n_max, dtype=torch.float32, device=index.kmin.device)
+    ix, pc = index.c(), plan.c()
+    st = _lib.kvs_selftest_scan_timeout(ctypes.byref(ix), ctypes.byref(pc), _ptr(nt), n_max,
+                                        _ptr(scores), wait_cycles, _ptr(dev_status), _stream(stream))
+    _check(st, "kvs_selftest_scan_timeout")
+
+
 def decode_step_workspace_size(R, G, H, n_max, k, B) -> int:
     return int(_lib.kvs_decode_step_workspace_size(R, G, H, n_max, k, B))
 
@@ -378,7 +454,7 @@ class DecodeStep:
     def __init__(self, index: FathomIndex, n, n_max: int, H: int, B: int, k: int, fullK, fullV,
                  slot_map=None, hotK=None, hotV=None, scale: float | None = None,
                  q_dtype=torch.float32, device=None):
-        dev = device or fullK.device
+        dev = device or index.kmin.device
         self.index, self.H, self.B, self.k, self.n_max = index, H, B, k, n_max
         R, G, D = index.R, index.G, index.D
         self.R, self.G, self.D = R, G, D
@@ -392,7 +468,10 @@ class DecodeStep:
         self.idx = torch.empty(R, G, k, dtype=torch.int32, device=dev)
         self.slots = torch.empty(R, G, k, dtype=torch.int32, device=dev)
         self.misses = torch.empty(R, G, dtype=torch.int32, device=dev)
-        wsb = decode_step_workspace_size(R, G, H, n_max, k, B)
+        # a full store in host memory (MappedHostStore) needs the staging too
+        self.full_on_host = isinstance(fullK, MappedHostStore)
+        wsb = (int(_lib.kvs_decode_step_workspace_size_host(R, G, H, n_max, k, B)) if self.full_on_host
+               else decode_step_workspace_size(R, G, H, n_max, k, B))
         self.ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
         self.q_dtype = KVS_BF16 if q_dtype == torch.bfloat16 else KVS_F32
         self._ix = index.c()

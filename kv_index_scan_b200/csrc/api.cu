@@ -4,6 +4,7 @@
 #include <cstring>
 
 #include "internal.cuh"
+#include "scan_core.cuh"
 
 namespace kvs {
 
@@ -144,6 +145,39 @@ kvs_status index_scan(const kvs_scan_args* a, float* scores, int32_t* dev_status
   return fail(KVS_EINVAL, "index_scan: unknown kind %d", a->kind);
 }
 
+kvs_status kvs_selftest_scan_timeout(const kvs_fathom_index* ix, const kvs_plan* plan, const int32_t* n,
+                                     int32_t n_max, float* scores, int64_t wait_cycles,
+                                     int32_t* dev_status, void* stream) {
+  kvs_status st = check_index(ix, n_max);
+  if (st != KVS_OK) return st;
+  st = check_plan(plan, ix->D);
+  if (st != KVS_OK) return st;
+  KVS_REQUIRE(n && scores && dev_status && n_max >= 1, KVS_EINVAL,
+              "kvs_selftest_scan_timeout: n, scores and dev_status are required, n_max >= 1");
+  KVS_REQUIRE(!ix->host_mapped && plan->B >= 1 && plan->B <= 144, KVS_EUNSUPPORTED,
+              "kvs_selftest_scan_timeout: an index in HBM and a plan of 1..144 planes");
+  KVS_REQUIRE(wait_cycles >= 1000 && wait_cycles <= 2000000000LL, KVS_EINVAL,
+              "kvs_selftest_scan_timeout: wait_cycles=%lld (1e3 .. 2e9)", static_cast<long long>(wait_cycles));
+  ScanParams p{};
+  p.planes = ix->planes;
+  p.W = ix->W;
+  p.RG = ix->R * ix->G;
+  p.Gheads = ix->G;
+  p.plane_idx = plan->plane_idx;
+  p.plane_w = plan->plane_w;
+  p.C = plan->C;
+  p.B = plan->B;
+  p.n = n;
+  p.n_max = n_max;
+  scan_schedule(plan->B, p.G, p.b, p.nsets);
+  p.scores = scores;
+  p.dev_status = dev_status;
+  p.wait_cycles = wait_cycles;
+  p.withhold_arrive = 1;
+  st = fathom_scan_lut_launch(p, static_cast<cudaStream_t>(stream));
+  return st == KVS_OK ? ok() : st;
+}
+
 size_t kvs_topk_workspace_size(int32_t R, int32_t G, int32_t n_max, int32_t k, int32_t block) {
   return topk_ws_bytes(R, G, n_max, k, block);
 }
@@ -185,6 +219,27 @@ kvs_status sparse_gather(const int32_t* idx, int32_t k, const int32_t* slot_map,
   return st == KVS_OK ? ok() : st;
 }
 
+kvs_status kvs_append_token(const uint16_t* Knew, const uint16_t* Vnew, int32_t* n, int32_t R,
+                            int32_t G, int32_t D, int32_t n_max, uint32_t* planes, int32_t W,
+                            const float* kmin, const float* kstep, uint16_t* fullK, uint16_t* fullV,
+                            int32_t* slot_map, const int32_t* hot_slot, int32_t* hot_tok,
+                            uint16_t* hotK, uint16_t* hotV, int32_t S, int32_t* dev_status,
+                            void* stream) {
+  KVS_REQUIRE(Knew && Vnew && n && planes && kmin && kstep && fullK && fullV, KVS_EINVAL,
+              "kvs_append_token: null pointer argument");
+  KVS_REQUIRE(R >= 1 && G >= 1 && G <= 8 && n_max >= 1, KVS_EINVAL,
+              "kvs_append_token: R=%d G=%d (1..8) n_max=%d", R, G, n_max);
+  KVS_REQUIRE(D == kD, KVS_EUNSUPPORTED, "kvs_append_token: D=%d (only 128 is built)", D);
+  KVS_REQUIRE(W >= 4 && W % 4 == 0 && 32LL * W >= n_max, KVS_EINVAL,
+              "kvs_append_token: W=%d must be a multiple of 4 with 32*W >= n_max=%d", W, n_max);
+  KVS_REQUIRE(!hot_slot || (slot_map && hot_tok && hotK && hotV && S >= 1), KVS_EINVAL,
+              "kvs_append_token: hot_slot needs slot_map, hot_tok, hotK, hotV and S >= 1");
+  kvs_status st = append_token_launch(Knew, Vnew, n, R, G, n_max, planes, W, kmin, kstep, fullK, fullV,
+                                      slot_map, hot_slot, hot_tok, hotK, hotV, S, dev_status,
+                                      static_cast<cudaStream_t>(stream));
+  return st == KVS_OK ? ok() : st;
+}
+
 size_t kvs_attn_workspace_size(int32_t R, int32_t G, int32_t H, int32_t k) {
   return attn_ws_bytes(R * G, H, k);
 }
@@ -216,6 +271,11 @@ kvs_status sparse_decode_attn(const void* q, int32_t q_dtype, const uint16_t* K,
   kvs_status st = attn_launch(q, q_dtype == KVS_BF16, src, R * G, H, scale, out, lse, ws,
                               static_cast<cudaStream_t>(stream));
   return st == KVS_OK ? ok() : st;
+}
+
+size_t kvs_decode_step_workspace_size_host(int32_t R, int32_t G, int32_t H, int32_t n_max, int32_t k,
+                                           int32_t B) {
+  return decode_ws_bytes_host(R, G, H, n_max, k, B);
 }
 
 size_t kvs_decode_step_workspace_size(int32_t R, int32_t G, int32_t H, int32_t n_max, int32_t k,
@@ -252,8 +312,14 @@ static kvs_status decode_step_checked(const kvs_decode_args* a, void* ws, size_t
   } else {
     KVS_REQUIRE(a->ix->R >= 1 && a->ix->G >= 1, KVS_EINVAL, "decode_step: index R/G");
   }
-  const size_t need = decode_ws_bytes(a->ix->R, a->ix->G, a->H, a->n_max, a->k,
-                                      a->plan ? a->plan->B : 0);
+  // a full store in host memory also needs the staging of the fetched misses
+  const bool host_full = a->fullK && host_resident(a->fullK);
+  KVS_REQUIRE(!host_full || host_resident(a->fullV), KVS_EINVAL,
+              "decode_step: fullK is host memory but fullV is not");
+  const size_t need = host_full ? decode_ws_bytes_host(a->ix->R, a->ix->G, a->H, a->n_max, a->k,
+                                                       a->plan ? a->plan->B : 0)
+                                : decode_ws_bytes(a->ix->R, a->ix->G, a->H, a->n_max, a->k,
+                                                  a->plan ? a->plan->B : 0);
   KVS_REQUIRE(ws && ws_bytes >= need, KVS_EWORKSPACE, "decode_step: workspace %zu < %zu bytes",
               ws_bytes, need);
   kvs_status st = decode_step_run(a, ws, dev_status, static_cast<cudaStream_t>(stream), ev);

@@ -92,6 +92,13 @@ __device__ __forceinline__ void split_bf16(float x, float y, uint32_t& hi, uint3
 // the staged / full store, c <= -2 hot slot -2 - c.
 __device__ __forceinline__ int row_code(const RowSrc& src, int u, int j) {
   if (j >= src.k) return -1;
+  if (src.mode == kRowsSlotStaged) {  // misses were fetched to staging row j
+    const int32_t* irow =
+        src.idx + (src.idx_shared ? static_cast<size_t>(u / src.G) : static_cast<size_t>(u)) * src.k;
+    const int i = __ldg(irow + j);
+    const int sl = __ldg(src.slots + static_cast<size_t>(u) * src.k + j);
+    return i < 0 ? -1 : (sl >= 0 ? -2 - sl : j);
+  }
   if (src.mode == kRowsStaged) {
     const int ke = src.k_eff ? src.k_eff[u] : src.k;
     return j < ke ? j : -1;
@@ -161,8 +168,8 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnBlocksPerSM) sparse_attn_ke
   }
 
   // row bases of this (r, g): staged rows are [u][k], full-store rows [u][n_max]
-  const size_t full_rows = src.mode == kRowsStaged ? static_cast<size_t>(src.k)
-                                                   : static_cast<size_t>(src.n_max);
+  const size_t full_rows = (src.mode == kRowsStaged || src.mode == kRowsSlotStaged)
+                               ? static_cast<size_t>(src.k) : static_cast<size_t>(src.n_max);
   const uint16_t* fK = src.K + static_cast<size_t>(u) * full_rows * kD;
   const uint16_t* fV = src.V + static_cast<size_t>(u) * full_rows * kD;
   const uint16_t* hK = src.hotK ? src.hotK + static_cast<size_t>(u) * src.S * kD : fK;

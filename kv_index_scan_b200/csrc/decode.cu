@@ -53,6 +53,16 @@ size_t decode_ws_bytes(int R, int G, int H, int n_max, int k, int B) {
   return c.used;
 }
 
+// With the full K/V store in host memory: the above, then the staging
+// buffers of the fetched misses (K and V, [RG][k][D] each).
+size_t decode_ws_bytes_host(int R, int G, int H, int n_max, int k, int B) {
+  WsCarver c(nullptr);
+  c.take<unsigned char>(decode_ws_bytes(R, G, H, n_max, k, B));
+  c.take<uint16_t>(static_cast<size_t>(R) * G * k * kD);
+  c.take<uint16_t>(static_cast<size_t>(R) * G * k * kD);
+  return c.used;
+}
+
 kvs_status decode_step_run(const kvs_decode_args* a, void* ws, int32_t* dev_status,
                            cudaStream_t s, cudaEvent_t const* ev) {
   const int R = a->ix->R, G = a->ix->G, RG = R * G;
@@ -120,8 +130,23 @@ kvs_status decode_step_run(const kvs_decode_args* a, void* ws, int32_t* dev_stat
   mark(3);
   RowSrc src{};
   src.mode = a->slot_map ? kRowsSlot : kRowsDirect;
-  src.K = a->fullK;
-  src.V = a->fullV;
+  if (host_resident(a->fullK)) {
+    // the full store lives in host memory: bring the misses into HBM first
+    WsCarver h(ws);
+    h.take<unsigned char>(decode_ws_bytes(R, G, a->H, a->n_max, a->k, a->plan ? a->plan->B : 0));
+    uint16_t* stageK = h.take<uint16_t>(static_cast<size_t>(RG) * a->k * kD);
+    uint16_t* stageV = h.take<uint16_t>(static_cast<size_t>(RG) * a->k * kD);
+    st = fetch_misses_launch(sel, shared, G, a->k, slots, a->fullK, a->fullV, a->n_max, RG, stageK,
+                             stageV, s);
+    if (st != KVS_OK) return st;
+    src.mode = kRowsSlotStaged;
+    src.K = stageK;
+    src.V = stageV;
+  }
+  if (src.mode != kRowsSlotStaged) {
+    src.K = a->fullK;
+    src.V = a->fullV;
+  }
   src.hotK = a->hotK;
   src.hotV = a->hotV;
   src.idx = sel;

@@ -7,7 +7,10 @@
 namespace kvs {
 
 // ---- attention row sources (attn.cu) ----
-enum RowMode { kRowsStaged = 0, kRowsSlot = 1, kRowsDirect = 2 };
+// kRowsSlotStaged: hits from the hot slots, misses from a staging buffer
+// [RG][k][D] at the entry's position j (the rows fetched from a full store in
+// host memory, fetch.cu)
+enum RowMode { kRowsStaged = 0, kRowsSlot = 1, kRowsDirect = 2, kRowsSlotStaged = 3 };
 
 struct RowSrc {
   int mode;
@@ -66,6 +69,16 @@ kvs_status attn_launch_fit(const void* q, int q_bf16, const RowSrc& src, int RG,
                            float scale, float* out, float* lse, float* part, size_t part_bytes,
                            size_t* need, cudaStream_t s);
 size_t decode_ws_bytes(int R, int G, int H, int n_max, int k, int B);
+bool host_resident(const void* p);
+kvs_status fetch_misses_launch(const int32_t* idx, int idx_shared, int G, int k, const int32_t* slots,
+                               const uint16_t* fullK, const uint16_t* fullV, int n_max, int RG,
+                               uint16_t* stageK, uint16_t* stageV, cudaStream_t s);
+size_t decode_ws_bytes_host(int R, int G, int H, int n_max, int k, int B);
+kvs_status append_token_launch(const uint16_t* Knew, const uint16_t* Vnew, int32_t* n, int R, int G,
+                               int n_max, uint32_t* planes, int W, const float* kmin, const float* kstep,
+                               uint16_t* fullK, uint16_t* fullV, int32_t* slot_map, const int32_t* hot_slot,
+                               int32_t* hot_tok, uint16_t* hotK, uint16_t* hotV, int S, int32_t* dev_status,
+                               cudaStream_t s);
 kvs_status decode_step_run(const kvs_decode_args* a, void* ws, int32_t* dev_status,
                            cudaStream_t s,
                            cudaEvent_t const* ev = nullptr);

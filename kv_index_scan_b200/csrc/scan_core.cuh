@@ -41,6 +41,11 @@ struct ScanParams {
   int32_t* cand_idx;
   int32_t* cand_count;  // [RG][segs]
   uint32_t* cand_tau;   // [RG][segs] score key below which a segment's entries are not needed
+  // the bound of every wait in cycles (0: kWaitCycles), and a self-test switch:
+  // producer warp 0 of every block withholds its arrival on its first chunk,
+  // so that the consumers' wait for that chunk runs out (kvs_selftest_scan_timeout)
+  long long wait_cycles;
+  int withhold_arrive;
 };
 
 // Picks the lookup schedule for a budget of B planes: the fewest groups per
@@ -115,12 +120,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait on a phase: false when about one second passes without it.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Bounded wait on a phase: false when `limit` cycles (about one second by
+// default) pass without it.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
 }

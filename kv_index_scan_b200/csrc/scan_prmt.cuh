@@ -166,6 +166,8 @@ struct ScanCoreP {
     atomicExch(abort_flag, 1);
   }
 
+  __device__ long long wait_limit() const { return p.wait_cycles > 0 ? p.wait_cycles : kWaitCycles; }
+
   __device__ static void sync() { consumer_sync<kPWarps>(); }
 
   // Producer warp j (0..3) stages planes j, j + 4, j + 8, ... of every chunk.
@@ -176,7 +178,7 @@ struct ScanCoreP {
     int u = beg / p.chunks_per_row, c = beg % p.chunks_per_row, st = 0;
     uint32_t phase = 0u;  // parity of the slot's next empty phase to wait for
     for (int it = beg; it < end; ++it) {
-      if (it - beg >= nstage && !mbar_wait(&empty[st], phase)) {
+      if (it - beg >= nstage && !mbar_wait(&empty[st], phase, wait_limit())) {
         if (lane == 0) fail_timeout();
         break;
       }
@@ -204,8 +206,9 @@ struct ScanCoreP {
                          : "memory");
         }
       }
-      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(smem_addr(&full[st]))
-                   : "memory");
+      if (!(p.withhold_arrive && j == 0 && it == beg))
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(smem_addr(&full[st]))
+                     : "memory");
       if (++c == p.chunks_per_row) {
         c = 0;
         ++u;
@@ -397,7 +400,7 @@ struct ScanCoreP {
       const int nr = row_n;
 #pragma unroll
       for (int j = 0; j < kPKeys; ++j) acc[j] = row_C;
-      if (!dead && !mbar_wait(&full[st], phase)) {
+      if (!dead && !mbar_wait(&full[st], phase, wait_limit())) {
         fail_timeout();
         dead = true;
       }

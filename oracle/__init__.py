@@ -58,6 +58,7 @@ def _declare(L):
     L.oracle_topk_f32.restype = I32
     L.oracle_gather.argtypes = [P, I32, P, P, P, P, P, I32, P, P, P]
     L.oracle_gather.restype = I32
+    L.oracle_append_token.argtypes = [P, P, I64, I32, I32, P, P, P, P, P, P, I32, P, P, P]
     L.oracle_attention.argtypes = [P, I32, I32, P, P, I32, F64, P, P]
     L.oracle_lightning_scores.argtypes = [P, I64, I32, P, I32, P, P]
     L.oracle_block_max.argtypes = [P, I64, I32, P]
@@ -114,6 +115,24 @@ def build_index(K, D: int, W: int):
     kmin, kstep, kvar = (np.zeros(D, np.float32) for _ in range(3))
     lib().oracle_build_index(_p(K), n, D, W, _p(planes), _p(kmin), _p(kstep), _p(kvar))
     return planes, kmin, kstep, kvar
+
+
+def append_token(knew, vnew, i: int, planes, kmin, kstep, fullK, fullV, slot_map=None, slot: int = -1,
+                 hot_tok=None, hotK=None, hotV=None):
+    """O0b for one row, on copies: returns (planes, fullK, fullV, slot_map,
+    hot_tok, hotK, hotV) after writing token i (see oracle.cpp)."""
+    planes = _arr(planes, np.uint32).copy()
+    D, _, W = planes.shape
+    fullK = _arr(fullK, np.uint16).copy()
+    fullV = _arr(fullV, np.uint16).copy()
+    sm = None if slot_map is None else _arr(slot_map, np.int32).copy()
+    ht = None if hot_tok is None else _arr(hot_tok, np.int32).copy()
+    hK = None if hotK is None else _arr(hotK, np.uint16).copy()
+    hV = None if hotV is None else _arr(hotV, np.uint16).copy()
+    lib().oracle_append_token(_p(_arr(knew, np.uint16)), _p(_arr(vnew, np.uint16)), i, D, W, _p(planes),
+                              _p(_arr(kmin, np.float32)), _p(_arr(kstep, np.float32)), _p(fullK),
+                              _p(fullV), _p(sm), slot, _p(ht), _p(hK), _p(hV))
+    return planes, fullK, fullV, sm, ht, hK, hV
 
 
 def plan_bits(q, kvar, B: int):

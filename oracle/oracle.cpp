@@ -127,6 +127,54 @@ void oracle_build_index(const uint16_t* K, int64_t n, int32_t D, int32_t W, uint
 }
 
 // ---------------------------------------------------------------------------
+// O0b. Per-step write-back of one new token into a row [XMSPARSE, the request
+// lifecycle list: the KV generated at each step is written back; FATHOM,
+// abstract: the 4-bit bit-plane K copy]. Reading: the new key is coded with
+// the row's stored quantiser (m, s), not a re-fitted one -- u = floor((k-m)/s
+// + 1/2) in fp64, clamped to 0..15, s = 0 -> u = 0 -- and its four plane bits
+// at position i are set to u's bits (plane 0 = MSB); its K and V rows go to
+// the full store at i. With a hot slot (slot >= 0) the rows are also copied
+// into that slot, the slot's previous token (hot_tok[slot], -1 if none) leaves
+// the slot map and the new token takes the slot; without one the new token's
+// slot-map entry is -1. kmin, kstep and kvar are left unchanged.
+//   knew, vnew bf16 [D]; planes u32 [D][4][W]; full bf16 [n_max][D];
+//   slot_map [n_max], hot_tok [S], hot bf16 [S][D] (nullable when slot < 0).
+void oracle_append_token(const uint16_t* knew, const uint16_t* vnew, int64_t i, int32_t D, int32_t W,
+                         uint32_t* planes, const float* kmin, const float* kstep, uint16_t* fullK,
+                         uint16_t* fullV, int32_t* slot_map, int32_t slot, int32_t* hot_tok,
+                         uint16_t* hotK, uint16_t* hotV) {
+  for (int32_t c = 0; c < D; ++c) {
+    const double m = static_cast<double>(kmin[c]);
+    const double s = static_cast<double>(kstep[c]);
+    int64_t u = 0;
+    if (s != 0.0) {
+      const double x = std::floor((bf16_to_double(knew[c]) - m) / s + 0.5);
+      u = x < 0.0 ? 0 : (x > 15.0 ? 15 : static_cast<int64_t>(x));
+    }
+    for (int p = 0; p < 4; ++p) {
+      uint32_t& w = planes[(static_cast<size_t>(c) * 4 + p) * W + static_cast<size_t>(i / 32)];
+      const uint32_t bit = 1u << (i % 32);
+      w = ((u >> (3 - p)) & 1) ? (w | bit) : (w & ~bit);
+    }
+    fullK[static_cast<size_t>(i) * D + c] = knew[c];
+    fullV[static_cast<size_t>(i) * D + c] = vnew[c];
+    if (slot >= 0) {
+      hotK[static_cast<size_t>(slot) * D + c] = knew[c];
+      hotV[static_cast<size_t>(slot) * D + c] = vnew[c];
+    }
+  }
+  if (slot_map) {
+    if (slot >= 0) {
+      if (hot_tok[slot] >= 0) slot_map[hot_tok[slot]] = -1;
+      hot_tok[slot] = static_cast<int32_t>(i);
+      slot_map[i] = slot;
+    } else {
+      slot_map[i] = -1;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // O1. Per-query bit allocation [FATHOM, abstract: each query divides its bit
 // budget among the key channels by reverse water-filling, with each channel's
 // importance weighted by its variance]. Reading: one allocation per (request, KV head) for the summed

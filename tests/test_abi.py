@@ -88,3 +88,28 @@ def test_product_package_does_not_import_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "oracle.cpp" not in text, f
+
+
+def test_selftest_and_append_argument_checks(kvs):
+    """The failure-path self-test and the write-back refuse bad arguments on
+    the host, before any launch."""
+    L = kvs._lib
+    ix = kvs.FathomIndexC(16, 16, 16, 16, 1, 1, 128, 128, 0)
+    plan = kvs.PlanC(16, 16, 16, 16, 92)
+    # no status word, a wait bound out of range, an index in host memory
+    assert L.kvs_selftest_scan_timeout(ctypes.byref(ix), ctypes.byref(plan), 16, 4096, 16, 2000000,
+                                       None, None) == kvs.KVS_EINVAL
+    assert L.kvs_selftest_scan_timeout(ctypes.byref(ix), ctypes.byref(plan), 16, 4096, 16, 10,
+                                       16, None) == kvs.KVS_EINVAL
+    ixh = kvs.FathomIndexC(16, 16, 16, 16, 1, 1, 128, 128, 1)
+    assert L.kvs_selftest_scan_timeout(ctypes.byref(ixh), ctypes.byref(plan), 16, 4096, 16, 2000000,
+                                       16, None) == kvs.KVS_EUNSUPPORTED
+    # append: W too small for n_max, G out of range, a hot slot without a slot map
+    args = [16, 16, 16, 1, 1, 128, 4096, 16, 128, 16, 16, 16, 16, None, None, None, None, None, 0, None, None]
+    a = list(args); a[8] = 64
+    assert L.kvs_append_token(*a) == kvs.KVS_EINVAL
+    a = list(args); a[4] = 9
+    assert L.kvs_append_token(*a) == kvs.KVS_EINVAL
+    a = list(args); a[14] = 16
+    assert L.kvs_append_token(*a) == kvs.KVS_EINVAL
+    assert b"hot_slot" in L.kvs_last_error()

@@ -420,3 +420,135 @@ def test_decode_step_timed_matches_and_records_stages(kvs):
     assert all(t >= 0 for t in times) and times[1] > 0 and times[3] > 0
     with pytest.raises(ValueError):
         step.timed(q, ev[:3])
+
+
+# ----------------------------------------------------------------------------- write-back
+
+def test_append_token_matches_the_oracle(kvs):
+    """kvs_append_token against the oracle's append, row by row: two tokens
+    appended in turn to ragged rows (the second request starts one short of
+    n_max, so its second append is refused with KVS_EBOUNDS and leaves the row
+    as it was), with a hot slot for some rows (the previous occupant evicted)
+    and none for the others."""
+    R, G, S, n_max = 3, 2, 16, 5000
+    nl = [3000, n_max - 1, 1]
+    K, V, _ = synth.fathom_kv(R, G, D, nl, n_max=n_max, seed=51)
+    Knew, Vnew, _ = synth.fathom_kv(R, G, D, 2, seed=52)
+    W = kvs.plane_words(n_max)
+    ix = kvs.build_fathom_index(K.to(DEV), nl, W)
+    rng = np.random.default_rng(51)
+    slot_map = np.full((R, G, n_max), -1, np.int32)
+    hot_tok = np.full((R, G, S), -1, np.int32)
+    for r in range(R):
+        for g in range(G):
+            toks = rng.choice(nl[r], min(S // 2, nl[r]), replace=False)
+            hot_tok[r, g, : toks.size] = toks
+            slot_map[r, g, toks] = np.arange(toks.size)
+    hotK, hotV = synth.hot_rows(K, hot_tok), synth.hot_rows(V, hot_tok)
+    hot_slot = np.array([[2, -1], [15, 0], [-1, 1]], np.int32)
+    dK, dV = K.clone().to(DEV), V.clone().to(DEV)
+    d_sm, d_ht = torch.from_numpy(slot_map).to(DEV), torch.from_numpy(hot_tok).to(DEV)
+    d_hK, d_hV = hotK.clone().to(DEV), hotV.clone().to(DEV)
+    n = torch.tensor(nl, dtype=torch.int32, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    ref = dict(planes=_np(ix.planes).view(np.uint32).copy(), K=_np(K).view(np.uint16).copy(),
+               V=_np(V).view(np.uint16).copy(), sm=slot_map.copy(), ht=hot_tok.copy(),
+               hK=_np(hotK).view(np.uint16).copy(), hV=_np(hotV).view(np.uint16).copy())
+    kmin, kstep = _np(ix.kmin), _np(ix.kstep)
+    pos = list(nl)
+    for step in range(2):
+        kvs.append_token(ix, Knew[:, :, step].to(DEV), Vnew[:, :, step].to(DEV), n, dK, dV, d_sm,
+                         torch.from_numpy(hot_slot).to(DEV), d_ht, d_hK, d_hV, dev_status=st)
+        torch.cuda.synchronize()
+        for r in range(R):
+            if pos[r] >= n_max:
+                continue
+            for g in range(G):
+                out = oracle.append_token(Knew[r, g, step], Vnew[r, g, step], pos[r], ref["planes"][r, g],
+                                          kmin[r, g], kstep[r, g], ref["K"][r, g], ref["V"][r, g],
+                                          ref["sm"][r, g], int(hot_slot[r, g]), ref["ht"][r, g],
+                                          ref["hK"][r, g], ref["hV"][r, g])
+                for key, val in zip(["planes", "K", "V", "sm", "ht", "hK", "hV"], out):
+                    ref[key][r, g] = val
+            pos[r] += 1
+    assert int(st.item()) == kvs.KVS_EBOUNDS  # request 1 was full at the second step
+    assert n.cpu().tolist() == pos == [nl[0] + 2, n_max, 3]
+    assert np.array_equal(_np(ix.planes).view(np.uint32), ref["planes"])
+    assert np.array_equal(_np(dK).view(np.uint16), ref["K"]) and np.array_equal(_np(dV).view(np.uint16), ref["V"])
+    assert np.array_equal(_np(d_sm), ref["sm"]) and np.array_equal(_np(d_ht), ref["ht"])
+    assert np.array_equal(_np(d_hK).view(np.uint16), ref["hK"])
+    assert np.array_equal(_np(d_hV).view(np.uint16), ref["hV"])
+
+
+# ----------------------------------------------------------------------------- failure detection
+
+def test_scan_bounded_wait_runs_out_and_the_context_stays_usable(kvs):
+    """A producer warp of every block of the HBM scan withholds its arrival on
+    its first chunk (kvs_selftest_scan_timeout), with every wait bounded by
+    2e6 cycles: the consumers' wait runs out, KVS_ETIMEOUT reaches the status
+    word, the kernel returns within milliseconds, and the next decode step on
+    the same context is exact."""
+    import time
+    R, G, H, n, B, k = 2, 4, 4, 70000, 92, 2048
+    K, V, nl = synth.fathom_kv(R, G, D, n, seed=61)
+    q = synth.queries(R, G, H, D, seed=61).to(DEV)
+    ix = kvs.build_fathom_index(K.to(DEV), nl)
+    plan = kvs.fathom_plan_bits(q, ix, B)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    kvs.selftest_scan_timeout(ix, plan, nl, n, 2_000_000, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == kvs.KVS_ETIMEOUT
+    assert time.perf_counter() - t0 < 5.0
+    st2 = torch.zeros(1, dtype=torch.int32, device=DEV)
+    step = kvs.DecodeStep(ix, nl, n, H, B, k, K.to(DEV), V.to(DEV))
+    step(q, dev_status=st2)
+    sc = kvs.index_scan_fathom(ix, step.plan, nl, n, dev_status=st2)
+    torch.cuda.synchronize()
+    assert int(st2.item()) == kvs.KVS_OK
+    order = torch.sort(sc.cpu(), dim=2, descending=True, stable=True).indices[:, :, :k]
+    assert torch.equal(step.idx.cpu(), torch.sort(order, dim=2).values.to(torch.int32))
+
+
+# ----------------------------------------------------------------------------- host tier
+
+@pytest.mark.parametrize("miss", [0.2, 0.4, 1.0])
+def test_full_store_in_host_memory_equals_the_hbm_step(kvs, miss):
+    """The full K/V store in mapped pinned host memory: the step fetches only
+    the missing selected rows over the host link into HBM before the
+    attention. Its outputs equal those of the same step with the store in HBM,
+    bit for bit, at 20% and 40% misses and with no hot buffer at all (every
+    selected row a miss); a second layer reusing the selection (idx_in) too."""
+    R, G, H, n, B, k, S = 2, 4, 4, 30000, 92, 512, 1024
+    K, V, nl = synth.fathom_kv(R, G, D, [n, 21000], n_max=n, seed=71)
+    q = synth.queries(R, G, H, D, seed=71).to(DEV)
+    Kd, Vd = K.to(DEV), V.to(DEV)
+    ix = kvs.build_fathom_index(Kd, nl)
+    if miss < 1.0:
+        warm = kvs.DecodeStep(ix, nl, n, H, B, k, Kd, Vd)
+        warm(q)
+        torch.cuda.synchronize()
+        slot_map, hot_tok = synth.slot_map_from_selection(warm.idx.cpu().numpy(), nl, n, S, miss, seed=72)
+        sm, hK, hV = (torch.from_numpy(slot_map).to(DEV), synth.hot_rows(Kd, hot_tok),
+                      synth.hot_rows(Vd, hot_tok))
+    else:
+        sm = hK = hV = None
+    ref = kvs.DecodeStep(ix, nl, n, H, B, k, Kd, Vd, sm, hK, hV)
+    hostK, hostV = kvs.MappedHostStore(Kd), kvs.MappedHostStore(Vd)
+    step = kvs.DecodeStep(ix, nl, n, H, B, k, hostK, hostV, sm, hK, hV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    ref(q)
+    step(q, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for name in ("out", "lse", "idx", "slots", "misses"):
+        assert torch.equal(getattr(step, name), getattr(ref, name)), name
+    expect = round(miss * k) if miss < 1.0 else k
+    assert torch.all(step.misses == expect)
+    # a second layer of a group reusing the selection, store in host memory
+    q2 = synth.queries(R, G, H, D, seed=73).to(DEV)
+    o_ref = ref(q2, idx_in=ref.idx).clone()
+    o_host = step(q2, idx_in=ref.idx)
+    torch.cuda.synchronize()
+    assert torch.equal(o_host, o_ref)

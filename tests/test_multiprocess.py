@@ -69,3 +69,14 @@ def test_reference_arm_under_torchrun_prints_once_from_rank_zero():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_sparq_like_channel_choice():
+    """The SparQ-like comparison scan of the selection-quality diagnostic reads
+    the r channels of largest |qbar_c|, ties to the lower channel."""
+    sys.path.insert(0, ROOT)
+    import bench
+    qbar = torch.tensor([[0.5, -2.0, 1.0, 2.0, -1.0, 0.1]])
+    assert bench.sparq_channels(qbar, 3).tolist() == [[1, 2, 3]]
+    assert bench.sparq_channels(qbar, 4).tolist() == [[1, 2, 3, 4]]
+    assert bench.sparq_channels(torch.zeros(1, 5), 2).tolist() == [[0, 1]]

@@ -494,3 +494,65 @@ def test_shared_attention_batch_reads_each_requests_selection():
             assert np.array_equal(out2[r, g], out[r, g]) and np.array_equal(lse2[r, g], lse[r, g])
         else:
             assert not out2[r, g].any()
+
+
+# ----------------------------------------------------------------------------- O0b append
+
+def test_append_equals_the_build_over_the_longer_row():
+    """Appending a key that lies inside the row's per-channel range (so the
+    quantiser of the longer row is the same) gives exactly the planes that
+    building the index over the longer row gives."""
+    n = 700
+    K, V = _kv(n + 1, seed=41)
+    K[0, 0, n] = ((K[0, 0, :n].float().amax(0) + K[0, 0, :n].float().amin(0)) / 2).to(torch.bfloat16)
+    W = synth.plane_words(n + 1)
+    planes_n, kmin, kstep, _ = oracle.build_index(K[0, 0, :n], D, W)
+    planes_n1, kmin1, kstep1, _ = oracle.build_index(K[0, 0, : n + 1], D, W)
+    assert np.array_equal(kmin, kmin1) and np.array_equal(kstep, kstep1)
+    fullK = np.zeros((n + 1, D), np.uint16)
+    fullV = np.zeros((n + 1, D), np.uint16)
+    out = oracle.append_token(K[0, 0, n], V[0, 0, n], n, planes_n, kmin, kstep, fullK, fullV)
+    assert np.array_equal(out[0], planes_n1)
+    assert np.array_equal(out[1][n], K[0, 0, n].view(torch.int16).numpy().view(np.uint16))
+
+
+def test_append_copies_an_existing_keys_codes_and_clamps_outside_the_range():
+    n = 300
+    K, V = _kv(n, seed=42)
+    W = synth.plane_words(n + 3)
+    planes, kmin, kstep, _ = oracle.build_index(K[0, 0], D, W)
+    fullK = np.zeros((n + 3, D), np.uint16)
+    fullV = np.zeros((n + 3, D), np.uint16)
+    # a copy of key 17 gets key 17's codes
+    p1 = oracle.append_token(K[0, 0, 17], V[0, 0, 17], n, planes, kmin, kstep, fullK, fullV)[0]
+    u17, _ = _codes_from_planes(p1, n + 1)
+    assert np.array_equal(u17[:, n], u17[:, 17])
+    # far below every channel's minimum -> 0, far above its maximum -> 15
+    lo = torch.full((D,), -1e4, dtype=torch.bfloat16)
+    hi = torch.full((D,), 1e4, dtype=torch.bfloat16)
+    p2 = oracle.append_token(lo, lo, n + 1, p1, kmin, kstep, fullK, fullV)[0]
+    p3 = oracle.append_token(hi, hi, n + 2, p2, kmin, kstep, fullK, fullV)[0]
+    u, _ = _codes_from_planes(p3, n + 3)
+    assert np.all(u[:, n + 1] == 0) and np.all(u[:, n + 2] == 15)
+    assert np.array_equal(u[:, :n + 1], u17)  # earlier keys untouched
+
+
+def test_append_hot_slot_evicts_the_previous_token():
+    n, S = 100, 8
+    K, V = _kv(n + 1, seed=43)
+    W = synth.plane_words(n + 1)
+    planes, kmin, kstep, _ = oracle.build_index(K[0, 0, :n], D, W)
+    slot_map = np.full(n + 1, -1, np.int32)
+    hot_tok = np.full(S, -1, np.int32)
+    slot_map[5], hot_tok[3] = 3, 5
+    hotK = np.zeros((S, D), np.uint16)
+    hotV = np.zeros((S, D), np.uint16)
+    fullK = np.zeros((n + 1, D), np.uint16)
+    fullV = np.zeros((n + 1, D), np.uint16)
+    _, fK, _, sm, ht, hK, hV = oracle.append_token(K[0, 0, n], V[0, 0, n], n, planes, kmin, kstep, fullK,
+                                                   fullV, slot_map, 3, hot_tok, hotK, hotV)
+    assert sm[5] == -1 and sm[n] == 3 and ht[3] == n
+    assert np.array_equal(hK[3], fK[n]) and np.array_equal(hV[3], V[0, 0, n].view(torch.int16).numpy().view(np.uint16))
+    _, _, _, sm2, _, _, _ = oracle.append_token(K[0, 0, n], V[0, 0, n], n, planes, kmin, kstep, fullK, fullV,
+                                                slot_map, -1, hot_tok, hotK, hotV)
+    assert sm2[n] == -1 and sm2[5] == 3  # no slot: a miss, the hot buffer untouched
