@@ -157,8 +157,11 @@ kvs_status decode_step_run(const kvs_decode_args* a, void* ws, int32_t* dev_stat
   src.S = a->S;
   src.G = G;
   src.k = a->k;
+  // q may be read before the wait on the preceding kernel when this step ran
+  // the plan kernel: it waits for everything before the step before it lets
+  // the chain go on, and no kernel of the step writes q
   st = attn_launch(a->q, a->q_dtype == KVS_BF16, src, RG, a->H, a->scale, a->out, a->lse,
-                   attn_ws, s);
+                   attn_ws, s, /*q_early=*/a->idx_in == nullptr);
   if (st != KVS_OK) return st;
   mark(4);
   return KVS_OK;

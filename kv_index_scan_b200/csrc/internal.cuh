@@ -63,8 +63,10 @@ kvs_status select_slots_launch(const int32_t* idx, int idx_shared, int G, int k,
                                int32_t* misses, cudaStream_t s);
 void attn_split(int RG, int k, int& nsplit, int& rows_per_split);
 size_t attn_ws_bytes(int RG, int H, int k);
+// q_early: q may be read before the wait on the preceding kernel (no kernel of
+// the launch chain writes it).
 kvs_status attn_launch(const void* q, int q_bf16, const RowSrc& src, int RG, int H, float scale,
-                       float* out, float* lse, void* ws, cudaStream_t s);
+                       float* out, float* lse, void* ws, cudaStream_t s, bool q_early = false);
 kvs_status attn_launch_fit(const void* q, int q_bf16, const RowSrc& src, int RG, int H,
                            float scale, float* out, float* lse, float* part, size_t part_bytes,
                            size_t* need, cudaStream_t s);
