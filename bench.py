@@ -790,6 +790,7 @@ def lightning_entry(args, dist, peak, bf16_peak, peak_kind, with_cpu: bool) -> d
     dev = torch.device("cuda", torch.cuda.current_device())
     R, n, Hi, Dl, block, k, G, H = (c[x] for x in ("R", "n", "Hi", "Dl", "block", "k", "G", "H"))
     kidx, qidx, w, nl = synth.lightning_inputs(R, n, Hi=Hi, Dl=Dl, seed=3, device=dev)
+    nl_dev = torch.tensor(nl, dtype=torch.int32, device=dev)  # resident: no copy inside the step
     layers = []
     for layer in range(2):
         K, V, _ = synth.fathom_kv(R, G, 128, n, seed=40, layer=layer, device=dev)
@@ -805,10 +806,10 @@ def lightning_entry(args, dist, peak, bf16_peak, peak_kind, with_cpu: bool) -> d
     def pair(ev=None):
         if ev:
             ev[0].record(stream)
-        kvs.index_scan_lightning(kidx, qidx, w, nl, block=block, scores=bs)
+        kvs.index_scan_lightning(kidx, qidx, w, nl_dev, block=block, scores=bs)
         if ev:
             ev[1].record(stream)
-        kvs.topk_select(bs, nl, k, block=block, idx=idx)
+        kvs.topk_select(bs, nl_dev, k, block=block, idx=idx)
         if ev:
             ev[2].record(stream)
         for j, (q, st) in enumerate(layers):
@@ -840,8 +841,10 @@ def lightning_entry(args, dist, peak, bf16_peak, peak_kind, with_cpu: bool) -> d
            "pair_achieved_gbs": pair_bytes / (pair_ms / 1e3) / 1e9,
            "pair_frac_hbm": pair_bytes / (pair_ms / 1e3) / 1e9 / peak,
            "indexer_tflops": flops / (scan_ms / 1e3) / 1e12,
-           "indexer_frac_tensor": flops / (scan_ms / 1e3) / 1e12 / bf16_peak,
-           "roofline": {"bound": "hbm", "kernel": "lightning_scan (tcgen05 kind::f16)",
+           # the e4m3 contraction against the measured bf16 peak x 2 (the nominal
+           # fp8 : bf16 ratio); hi and lo query parts make two passes
+           "indexer_frac_tensor": 2 * flops / (scan_ms / 1e3) / 1e12 / (2 * bf16_peak),
+           "roofline": {"bound": "hbm", "kernel": "lightning_scan (tcgen05 kind::f8f6f4)",
                         "achieved": scan_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                         "frac": scan_gbs / peak, "traffic": None, "algorithmic_bytes": kbytes,
                         "ms": scan_ms},
@@ -952,6 +955,8 @@ def _run_row(args) -> dict:
         c = LIGHTNING
         R, n, Hi, Dl, block, k = (c[x] for x in ("R", "n", "Hi", "Dl", "block", "k"))
         sets = [synth.lightning_inputs(R, n, Hi, Dl, seed=3 + j, device=dev) for j in range(2)]
+        # request lengths resident on the device, so that no copy falls inside the timing
+        sets = [(kk, qq, ww, torch.tensor(nn, dtype=torch.int32, device=dev)) for kk, qq, ww, nn in sets]
         nb = (n + block - 1) // block
         bs = torch.empty(R, nb, dtype=torch.float32, device=dev)
         scan_ms = _time_ms(lambda i: kvs.index_scan_lightning(*sets[i & 1][:3], sets[i & 1][3],
@@ -971,6 +976,7 @@ def _run_row(args) -> dict:
     if args.row == "host-scan":
         R, G, n, B = 4, 8, 1048576, 92
         K, _, nl = synth.fathom_kv(R, G, 128, n, seed=2, device=dev, with_v=False)
+        nl = torch.tensor(nl, dtype=torch.int32, device=dev)  # resident: no copy inside the timing
         q = synth.queries(R, G, 4, 128, seed=2, device=dev)
         ix = kvs.build_fathom_index(K, nl)
         del K

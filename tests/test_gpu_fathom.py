@@ -82,6 +82,30 @@ def test_plan_bits_bit_exact(kvs, B):
             assert abs(float(_np(plan.C)[r, g]) - cref) <= tol
 
 
+@pytest.mark.parametrize("B", [1, 37, 92, 136, 300, 511])
+def test_plan_bits_bit_exact_with_tied_and_zero_weights(kvs, B):
+    """Channels with equal variances and queries with few distinct values give
+    many equal weights w_c (ties go to the lowest channel), constant channels
+    give w_c = 0, and weights 4x apart tie across bit positions."""
+    R, G, H, n = 1, 4, 4, 256
+    gen = torch.Generator().manual_seed(B)
+    base = torch.randn(n, generator=gen)
+    scale = torch.tensor([1.0, 2.0, 0.5, 0.0])[torch.randint(0, 4, (R, G, D), generator=gen)]
+    K = (base.view(1, 1, n, 1) * scale.view(R, G, 1, D)).to(torch.bfloat16).contiguous()
+    q = torch.tensor([-1.0, 0.5, 1.0, 2.0])[torch.randint(0, 4, (R, G, H, D), generator=gen)]
+    q[0, 3] = 0.0
+    q[0, 3, 0] = torch.pow(2.0, torch.randint(-3, 4, (D,), generator=gen).float())
+    ix = kvs.build_fathom_index(K.to(DEV), [n] * R)
+    plan = kvs.fathom_plan_bits(q.to(DEV), ix, B)
+    torch.cuda.synchronize()
+    kvar, t_gpu = _np(ix.kvar), _np(plan.t)
+    for g in range(G):
+        t, _ = oracle.plan_bits(q[0, g], kvar[0, g], B)
+        assert np.array_equal(t_gpu[0, g], t), g
+        pidx = _np(plan.plane_idx)[0, g, :B].view(np.uint16).astype(np.int64)
+        assert np.array_equal(pidx, [4 * c + p for c in range(D) for p in range(t[c])])
+
+
 # ----------------------------------------------------------------------------- a2 scan
 
 @pytest.mark.parametrize("B", [0, 1, 7, 33, 68, 72, 73, 92, 136, 144, 145, 300, 512])
