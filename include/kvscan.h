@@ -186,12 +186,18 @@ KVS_API kvs_status fathom_plan_bits(const float* q /* f32 [R][G][H][D] */, int32
  * KVS_SCAN_LIGHTNING [MINIMAX]: per request r and token i < n[r],
  *   S_i = sum_{h < Hi} w_h * max(0, q_h . k_i)
  *   with k_i = kidx e4m3 [R][n_max][Dl], q_h = qidx bf16 [R][Hi][Dl],
- *   w_h = widx f32 [R][Hi], computed on the tcgen05 tensor cores with f32
- *   accumulation. With block > 1 the output is the block score
+ *   w_h = widx f32 [R][Hi], computed on the tcgen05 tensor cores straight on
+ *   the e4m3 keys (kind::f8f6f4) with f32 accumulation. Each request's q is
+ *   scaled by a power of two and split into two e4m3 parts, hi and the
+ *   residual lo, whose sum is q exactly except for components more than 2^10
+ *   below the request's largest |q| (their bits below the e4m3 subnormal step
+ *   are rounded away). With block > 1 the output is the block score
  *   scores f32 [R][ceil(n_max/block)], b_j = max of S_i over the valid tokens
  *   of block j (-inf for blocks past n[r]); with block == 1 it is S itself,
- *   [R][n_max]. Dl must be 128, Hi a multiple of 16 up to 128, block 1 or a
- *   multiple of 32 up to 128.
+ *   [R][n_max]. Dl must be 128, Hi a multiple of 16 up to 128, block 1, 32,
+ *   64 or 128, kidx 16-byte aligned and R * n_max below 2^31 (KVS_EINVAL /
+ *   KVS_EUNSUPPORTED otherwise); KVS_ECUDA when the driver's tensor-map
+ *   encoder cannot be reached.
  * ------------------------------------------------------------------------- */
 typedef struct {
   int32_t kind;

@@ -25,11 +25,11 @@
 //    the next MMA (O[heads][dims] += P[heads][rows] V[rows][dims]); P is split
 //    into hi/lo bf16 parts the same way, V comes from ldmatrix.trans.
 //  * Online softmax per head inside the four lanes that hold it; the block's
-//    warps merge by log-sum-exp in shared memory. The blocks (splits) of one
-//    (r, g) form a thread-block cluster when there are at most 8 of them: each
-//    leaves its merged partial in its shared memory and the cluster's first
-//    block merges them through distributed shared memory. More splits write
-//    their partials to global memory for a second small kernel.
+//    warps merge by log-sum-exp in shared memory, and the blocks (splits) of
+//    one (r, g) in a second small kernel. (Merging the splits inside a
+//    thread-block cluster instead made the kernel faster alone but the decode
+//    step slower: a clustered launch lost the overlap with its neighbours that
+//    programmatic dependent launch gives the step's kernels.)
 #include <cuda_bf16.h>
 
 #include "internal.cuh"
@@ -44,7 +44,6 @@ constexpr int kAttnBlocksPerSM = 2;
 constexpr int kAttnStages = 3;
 constexpr int kTileRows = 16;
 constexpr int kSplitUnit = 64;                           // rows: the granularity of a split
-constexpr int kMaxClusterSplits = 8;                     // portable cluster size
 constexpr int kStageBytes = 2 * kTileRows * kD * 2;      // K and V of one tile, bf16
 constexpr int kAttnSmem = kAttnWarps * kAttnStages * kStageBytes;  // 96 KB
 
@@ -125,35 +124,13 @@ __device__ __forceinline__ int row_code(const RowSrc& src, int u, int j) {
   return i;
 }
 
-// Distributed shared memory of a cluster: the address of the same shared
-// variable in block `rank` of this block's cluster, and a 16-byte load from it.
-__device__ __forceinline__ uint32_t cluster_peer_addr(uint32_t local, int rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(local), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];\n"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
-// Every thread of every block of the cluster arrives; shared-memory writes
-// before it are visible to the cluster's reads after it.
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
-}
-
 // q_early: q is read before the wait on the preceding kernel (allowed when no
 // kernel of the chain writes q, as in the decode step, where q is its input).
-// cluster_merge: the nsplit blocks of one (r, g) are one cluster (nsplit <= 8).
 template <int H>
 __global__ void __launch_bounds__(kAttnThreads, kAttnBlocksPerSM) sparse_attn_kernel(
     const void* __restrict__ q, int q_bf16, RowSrc src, int nsplit, int rows_per_split,
     float scale_log2, float* __restrict__ out, float* __restrict__ lse,
-    float* __restrict__ part, int q_early, int cluster_merge) {
+    float* __restrict__ part, int q_early) {
   if (!q_early) pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(128) unsigned char attn_smem[];
@@ -353,8 +330,6 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnBlocksPerSM) sparse_attn_ke
     }
   }
   __syncthreads();
-  // the block's merged partial of head h, [M, L, -, -, acc[kD]] (cluster merge)
-  float* sm_part = sm_ml + kAttnWarps * H * 2;
   for (int h = warp; h < H; h += kAttnWarps) {
     float M = ninf;
 #pragma unroll
@@ -380,8 +355,7 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnBlocksPerSM) sparse_attn_ke
       if (lse && lane == 0)
         lse[static_cast<size_t>(u) * H + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : ninf;
     } else {
-      float* pp = cluster_merge ? sm_part + h * (kD + 4)
-                                : part + ((static_cast<size_t>(u) * nsplit + split) * H + h) * (kD + 4);
+      float* pp = part + ((static_cast<size_t>(u) * nsplit + split) * H + h) * (kD + 4);
       *reinterpret_cast<float4*>(pp + 4 + 4 * lane) = make_float4(acc[0], acc[1], acc[2], acc[3]);
       if (lane == 0) {
         pp[0] = M;
@@ -389,40 +363,6 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnBlocksPerSM) sparse_attn_ke
       }
     }
   }
-  if (!cluster_merge) return;
-  // The splits of (r, g) are the blocks of this cluster, rank = split. The
-  // first block merges head h in warp h, in split order (the arithmetic of
-  // attn_combine_kernel); the second barrier keeps every block's shared
-  // memory alive until those reads are done.
-  cluster_sync_all();
-  if (split == 0) {
-    for (int h = warp; h < H; h += kAttnWarps) {
-      const uint32_t mine = smem_u32(sm_part + h * (kD + 4));
-      float M = ninf;
-      for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, ld_cluster_f4(cluster_peer_addr(mine, sp)).x);
-      float L = 0.f;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (M != ninf) {
-        for (int sp = 0; sp < nsplit; ++sp) {
-          const uint32_t pp = cluster_peer_addr(mine, sp);
-          const float4 ml = ld_cluster_f4(pp);
-          const float w = exp2f(ml.x - M);
-          L += ml.y * w;
-          const float4 v = ld_cluster_f4(pp + 16 + 16 * lane);
-          acc.x += w * v.x;
-          acc.y += w * v.y;
-          acc.z += w * v.z;
-          acc.w += w * v.w;
-        }
-      }
-      const float inv = L > 0.f ? 1.f / L : 0.f;
-      *reinterpret_cast<float4*>(out + (static_cast<size_t>(u) * H + h) * kD + 4 * lane) =
-          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-      if (lse && lane == 0)
-        lse[static_cast<size_t>(u) * H + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : ninf;
-    }
-  }
-  cluster_sync_all();
 }
 
 // Merge of the splits of one (r, g): warp h merges head h by log-sum-exp.
@@ -462,11 +402,9 @@ kvs_status launch_h(const void* q, int q_bf16, const RowSrc& src, int RG, int ns
                     float scale_log2, float* out, float* lse, float* part, int q_early, cudaStream_t s) {
   cudaFuncSetAttribute(sparse_attn_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        kAttnSmem);
-  const int cluster = nsplit > 1 && nsplit <= kMaxClusterSplits ? nsplit : 1;
-  launch_chained_cluster(sparse_attn_kernel<H>, dim3(RG * nsplit), dim3(kAttnThreads), kAttnSmem, s, cluster, q,
-                 q_bf16, src, nsplit, rps, scale_log2, out, lse, part, q_early, cluster > 1 ? 1 : 0);
-  if (nsplit > 1 && cluster == 1)
-    launch_chained(attn_combine_kernel, dim3(RG), dim3(H * 32), 0, s, part, nsplit, H, out, lse);
+  launch_chained(sparse_attn_kernel<H>, dim3(RG * nsplit), dim3(kAttnThreads), kAttnSmem, s, q, q_bf16, src,
+                 nsplit, rps, scale_log2, out, lse, part, q_early);
+  if (nsplit > 1) launch_chained(attn_combine_kernel, dim3(RG), dim3(H * 32), 0, s, part, nsplit, H, out, lse);
   return check_launch("sparse_decode_attn");
 }
 
