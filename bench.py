@@ -88,6 +88,9 @@ TRAFFIC: dict = {
     # R=8 capture of fathom_scan_prmt_kernel: 96.56 MB read + 9.77 MB written
     # per launch (the rest of its scores leave L2 later), x2 for R=16
     ("qwen3-8b-128k", 92, "fathom_scan_prmt"): 2 * (96_558_080 + 9_770_752),
+    # full capture of lightning_scan_kernel<4> at 32 x 80000 tokens x 64 heads
+    # (the bench's own workload): 328.70 MB read + 4.64 MB written per launch
+    ("minimax-lightning-32x80000", 64, "lightning_scan"): 328_696_832 + 4_638_720,
 }
 
 
@@ -846,7 +849,9 @@ def lightning_entry(args, dist, peak, bf16_peak, peak_kind, with_cpu: bool) -> d
            "indexer_frac_tensor": 2 * flops / (scan_ms / 1e3) / 1e12 / (2 * bf16_peak),
            "roofline": {"bound": "hbm", "kernel": "lightning_scan (tcgen05 kind::f8f6f4)",
                         "achieved": scan_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                        "frac": scan_gbs / peak, "traffic": None, "algorithmic_bytes": kbytes,
+                        "frac": scan_gbs / peak,
+                        "traffic": TRAFFIC.get(("minimax-lightning-32x80000", Hi, "lightning_scan")),
+                        "algorithmic_bytes": kbytes,
                         "ms": scan_ms},
            "clocks": reg.clocks()}
     if with_cpu and (dist is None or dist.get_rank() == 0):
