@@ -24,6 +24,13 @@
 //  * P.V: the logit accumulators are, element for element, the A operand of
 //    the next MMA (O[heads][dims] += P[heads][rows] V[rows][dims]); P is split
 //    into hi/lo bf16 parts the same way, V comes from ldmatrix.trans.
+//  * With H <= 4 the 16 MMA rows are the tile's tokens instead and the 8
+//    columns the heads' hi and lo query parts (4 + 4): S[rows][cols] = K Q^T
+//    takes 8 MMAs per tile instead of 16, and O^T[dims][cols] += V^T P^T
+//    8 instead of 16, with V^T from ldmatrix.trans and P^T from the logit
+//    accumulators by movmatrix.trans (hi parts in the columns of lanes
+//    c < 2, lo parts in those of c >= 2). A head's logit is the sum of its hi
+//    and lo columns; O's two halves are added at the end.
 //  * Online softmax per head inside the four lanes that hold it; the block's
 //    warps merge by log-sum-exp in shared memory, and the blocks (splits) of
 //    one (r, g) in a second small kernel. (Merging the splits inside a
@@ -78,6 +85,13 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       "{%8, %9}, {%0, %1, %2, %3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// The 8x8 b16 matrix held one row pair per lane (lane 4r + c: row r, columns
+// 2c, 2c + 1), transposed in the same layout.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
 }
 // Two floats as bf16 (round to nearest even), x in the low half.
 __device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
@@ -143,32 +157,44 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnBlocksPerSM) sparse_attn_ke
   const int j_end = min(src.k, j_begin + rows_per_split);
   const uint32_t ring = smem_u32(attn_smem) + warp * kAttnStages * kStageBytes;
 
-  // A operand of the logits MMA: row g = q_hi of head g, row g + 8 = q_lo
-  uint32_t qa[8][4];
+  constexpr bool kTok = H <= 4;  // tokens as the MMA's M dimension
+  // kTok: B operand of the logits MMA, column g = head g & 3, its hi part for
+  // g < 4 and its lo part for g >= 4, over dims 16 ks + 2 tq (+1, +8, +9).
+  // Otherwise: A operand, row g = q_hi of head g, row g + 8 = q_lo.
+  uint32_t qa[8][kTok ? 2 : 4];
+  auto q_pair = [&](int head, int d0, float& x, float& y) {
+    x = 0.f;
+    y = 0.f;
+    if (head < H) {
+      const size_t off = (static_cast<size_t>(u) * H + head) * kD + d0;
+      if (q_bf16) {
+        const uint16_t* qq = reinterpret_cast<const uint16_t*>(q) + off;
+        x = bf16_bits_to_float(qq[0]);
+        y = bf16_bits_to_float(qq[1]);
+      } else {
+        const float* qq = reinterpret_cast<const float*>(q) + off;
+        x = qq[0];
+        y = qq[1];
+      }
+      x *= scale_log2;
+      y *= scale_log2;
+    }
+  };
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int d0 = 16 * ks + 8 * half + 2 * tq;
-      float x = 0.f, y = 0.f;
-      if (g < H) {
-        const size_t off = (static_cast<size_t>(u) * H + g) * kD + d0;
-        if (q_bf16) {
-          const uint16_t* qq = reinterpret_cast<const uint16_t*>(q) + off;
-          x = bf16_bits_to_float(qq[0]);
-          y = bf16_bits_to_float(qq[1]);
-        } else {
-          const float* qq = reinterpret_cast<const float*>(q) + off;
-          x = qq[0];
-          y = qq[1];
-        }
-        x *= scale_log2;
-        y *= scale_log2;
-      }
+      float x, y;
+      q_pair(kTok ? (g & 3) : g, d0, x, y);
       uint32_t hi, lo;
       split_bf16(x, y, hi, lo);
-      qa[ks][2 * half] = hi;
-      qa[ks][2 * half + 1] = lo;
+      if constexpr (kTok) {
+        qa[ks][half] = g < 4 ? hi : lo;
+      } else {
+        qa[ks][2 * half] = hi;
+        qa[ks][2 * half + 1] = lo;
+      }
     }
   }
   if (q_early) pdl_wait();
@@ -214,12 +240,15 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnBlocksPerSM) sparse_attn_ke
     return vm;
   };
 
-  float o[16][4];
+  float o[kTok ? 8 : 16][4];
 #pragma unroll
-  for (int d = 0; d < 16; ++d)
+  for (int d = 0; d < (kTok ? 8 : 16); ++d)
 #pragma unroll
     for (int e = 0; e < 4; ++e) o[d][e] = 0.f;
   float m_run = ninf, l_run = 0.f;  // of head g, shared by the four lanes of group g
+  // kTok: this lane's heads hA = 2 (tq & 1) and hA + 1; l is the lane's part
+  // (tokens g and g + 8 of each tile), summed over the lanes at the end
+  float mA = ninf, mB = ninf, lA = 0.f, lB = 0.f;
 
   // prologue: tiles 0 and 1 in flight, the codes of tiles 2..5 on their way
   // (row locations are fetched four tiles ahead of their copies)
@@ -244,70 +273,134 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnBlocksPerSM) sparse_attn_ke
     const uint32_t kst = ring + st * kStageBytes;
     const uint32_t vst = kst + kTileRows * kD * 2;
 
+    if constexpr (kTok) {
+      // ---- S[tokens][cols] = K Q^T: A = the K tile (ldmatrix), B = q ----
+      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t a[4];
+        const int row = lane & 15;
+        const int chunk = 2 * ks + (lane >> 4);
+        ldsm_x4(kst + row * (kD * 2) + ((chunk ^ (row & 7)) << 4), a);
+        mma_bf16(sc, a, qa[ks][0], qa[ks][1]);
+      }
+      // logits of heads hA, hA + 1 for tokens g and g + 8: hi column + lo column
+      float s4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s4[e] = sc[e] + __shfl_xor_sync(0xFFFFFFFFu, sc[e], 2);
+      const bool vg = (vm0 >> g) & 1u, vg8 = (vm0 >> (g + 8)) & 1u;
+      s4[0] = vg ? s4[0] : ninf;
+      s4[1] = vg ? s4[1] : ninf;
+      s4[2] = vg8 ? s4[2] : ninf;
+      s4[3] = vg8 ? s4[3] : ninf;
+      float mxA = fmaxf(s4[0], s4[2]), mxB = fmaxf(s4[1], s4[3]);
+#pragma unroll
+      for (int d = 4; d < 32; d <<= 1) {
+        mxA = fmaxf(mxA, __shfl_xor_sync(0xFFFFFFFFu, mxA, d));
+        mxB = fmaxf(mxB, __shfl_xor_sync(0xFFFFFFFFu, mxB, d));
+      }
+      const float nA = fmaxf(mA, mxA), nB = fmaxf(mB, mxB);
+      const bool noneA = nA == ninf, noneB = nB == ninf;
+      const float alA = noneA ? 1.f : exp2f(mA - nA), alB = noneB ? 1.f : exp2f(mB - nB);
+      float p4[4];
+      p4[0] = noneA ? 0.f : exp2f(s4[0] - nA);
+      p4[2] = noneA ? 0.f : exp2f(s4[2] - nA);
+      p4[1] = noneB ? 0.f : exp2f(s4[1] - nB);
+      p4[3] = noneB ? 0.f : exp2f(s4[3] - nB);
+      lA = lA * alA + (p4[0] + p4[2]);
+      lB = lB * alB + (p4[1] + p4[3]);
+      mA = nA;
+      mB = nB;
+      if (!__all_sync(0xFFFFFFFFu, alA == 1.f && alB == 1.f)) {
+#pragma unroll
+        for (int d = 0; d < 8; ++d) {
+          o[d][0] *= alA;
+          o[d][2] *= alA;
+          o[d][1] *= alB;
+          o[d][3] *= alB;
+        }
+      }
+      // ---- O^T[dims][cols] += V^T P^T: P^T by movmatrix, V^T by ldmatrix.trans ----
+      uint32_t h01, l01, h23, l23;
+      split_bf16(p4[0], p4[1], h01, l01);
+      split_bf16(p4[2], p4[3], h23, l23);
+      const uint32_t b0 = movmatrix_trans(tq < 2 ? h01 : l01);
+      const uint32_t b1 = movmatrix_trans(tq < 2 ? h23 : l23);
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        uint32_t a[4];
+        const int mi = lane >> 3;
+        const int tok = (lane & 7) + 8 * (mi >> 1);
+        const int chunk = 2 * mt + (mi & 1);
+        ldsm_x4_trans(vst + tok * (kD * 2) + ((chunk ^ (tok & 7)) << 4), a);
+        mma_bf16(o[mt], a, b0, b1);
+      }
+    } else {
     // ---- logits of the tile's 16 rows (two n-tiles of 8) ----
-    float sc[2][4];
+      float sc[2][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
+        for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      uint32_t b[4];
-      const int row = (lane & 7) + ((lane >> 4) << 3);
-      const int chunk = 2 * ks + ((lane >> 3) & 1);
-      ldsm_x4(kst + row * (kD * 2) + ((chunk ^ (row & 7)) << 4), b);
-      mma_bf16(sc[0], qa[ks], b[0], b[1]);
-      mma_bf16(sc[1], qa[ks], b[2], b[3]);
-    }
-    // ---- online softmax of head g over rows n = 8 nt + 2 tq + e ----
-    float s[2][2];
-    float mx = ninf;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int n = 8 * nt + 2 * tq + e;
-        const float v = sc[nt][e] + sc[nt][e + 2];
-        s[nt][e] = ((vm0 >> n) & 1u) ? v : ninf;
-        mx = fmaxf(mx, s[nt][e]);
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t b[4];
+        const int row = (lane & 7) + ((lane >> 4) << 3);
+        const int chunk = 2 * ks + ((lane >> 3) & 1);
+        ldsm_x4(kst + row * (kD * 2) + ((chunk ^ (row & 7)) << 4), b);
+        mma_bf16(sc[0], qa[ks], b[0], b[1]);
+        mma_bf16(sc[1], qa[ks], b[2], b[3]);
       }
-    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
-    const float m_new = fmaxf(m_run, mx);
-    const bool none = m_new == ninf;
-    const float alpha = none ? 1.f : exp2f(m_run - m_new);
-    float p[2][2];
-    float ps = 0.f;
+      // ---- online softmax of head g over rows n = 8 nt + 2 tq + e ----
+      float s[2][2];
+      float mx = ninf;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        p[nt][e] = none ? 0.f : exp2f(s[nt][e] - m_new);
-        ps += p[nt][e];
+        for (int e = 0; e < 2; ++e) {
+          const int n = 8 * nt + 2 * tq + e;
+          const float v = sc[nt][e] + sc[nt][e + 2];
+          s[nt][e] = ((vm0 >> n) & 1u) ? v : ninf;
+          mx = fmaxf(mx, s[nt][e]);
+        }
+      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
+      const float m_new = fmaxf(m_run, mx);
+      const bool none = m_new == ninf;
+      const float alpha = none ? 1.f : exp2f(m_run - m_new);
+      float p[2][2];
+      float ps = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          p[nt][e] = none ? 0.f : exp2f(s[nt][e] - m_new);
+          ps += p[nt][e];
+        }
+      ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 1);
+      ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 2);
+      l_run = l_run * alpha + ps;
+      m_run = m_new;
+      if (!__all_sync(0xFFFFFFFFu, alpha == 1.f)) {
+#pragma unroll
+        for (int d = 0; d < 16; ++d)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[d][e] *= alpha;
       }
-    ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 1);
-    ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 2);
-    l_run = l_run * alpha + ps;
-    m_run = m_new;
-    if (!__all_sync(0xFFFFFFFFu, alpha == 1.f)) {
+      // ---- P.V: P (hi/lo split) is the A operand, V from ldmatrix.trans ----
+      uint32_t pa[4];
+      split_bf16(p[0][0], p[0][1], pa[0], pa[1]);
+      split_bf16(p[1][0], p[1][1], pa[2], pa[3]);
 #pragma unroll
-      for (int d = 0; d < 16; ++d)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[d][e] *= alpha;
-    }
-    // ---- P.V: P (hi/lo split) is the A operand, V from ldmatrix.trans ----
-    uint32_t pa[4];
-    split_bf16(p[0][0], p[0][1], pa[0], pa[1]);
-    split_bf16(p[1][0], p[1][1], pa[2], pa[3]);
-#pragma unroll
-    for (int d2 = 0; d2 < 8; ++d2) {
-      uint32_t b[4];
-      const int mi = lane >> 3;
-      const int row = (lane & 7) + 8 * (mi & 1);
-      const int chunk = 2 * d2 + (mi >> 1);
-      ldsm_x4_trans(vst + row * (kD * 2) + ((chunk ^ (row & 7)) << 4), b);
-      mma_bf16(o[2 * d2], pa, b[0], b[1]);
-      mma_bf16(o[2 * d2 + 1], pa, b[2], b[3]);
+      for (int d2 = 0; d2 < 8; ++d2) {
+        uint32_t b[4];
+        const int mi = lane >> 3;
+        const int row = (lane & 7) + 8 * (mi & 1);
+        const int chunk = 2 * d2 + (mi >> 1);
+        ldsm_x4_trans(vst + row * (kD * 2) + ((chunk ^ (row & 7)) << 4), b);
+        mma_bf16(o[2 * d2], pa, b[0], b[1]);
+        mma_bf16(o[2 * d2 + 1], pa, b[2], b[3]);
+      }
     }
     __syncwarp();  // the stage is refilled by the next iteration's copies
     vm0 = vm1;
@@ -319,7 +412,43 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnBlocksPerSM) sparse_attn_ke
   // ---- merge the block's warps by log-sum-exp (the ring is free now) ----
   float* sm_o = reinterpret_cast<float*>(attn_smem);  // [warps][H][kD]
   float* sm_ml = sm_o + kAttnWarps * H * kD;          // [warps][H][2]
-  if (g < H) {
+  if constexpr (kTok) {
+    // O = the hi columns + the lo columns (lanes tq and tq ^ 2); l over the
+    // lanes' tokens
+#pragma unroll
+    for (int d = 0; d < 8; ++d)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[d][e] += __shfl_xor_sync(0xFFFFFFFFu, o[d][e], 2);
+#pragma unroll
+    for (int d = 4; d < 32; d <<= 1) {
+      lA += __shfl_xor_sync(0xFFFFFFFFu, lA, d);
+      lB += __shfl_xor_sync(0xFFFFFFFFu, lB, d);
+    }
+    const int hA = 2 * (tq & 1), hB = hA + 1;
+    if (tq < 2) {
+#pragma unroll
+      for (int d = 0; d < 8; ++d) {
+        if (hA < H) {
+          sm_o[(warp * H + hA) * kD + 16 * d + g] = o[d][0];
+          sm_o[(warp * H + hA) * kD + 16 * d + g + 8] = o[d][2];
+        }
+        if (hB < H) {
+          sm_o[(warp * H + hB) * kD + 16 * d + g] = o[d][1];
+          sm_o[(warp * H + hB) * kD + 16 * d + g + 8] = o[d][3];
+        }
+      }
+      if (g == 0) {
+        if (hA < H) {
+          sm_ml[(warp * H + hA) * 2] = mA;
+          sm_ml[(warp * H + hA) * 2 + 1] = lA;
+        }
+        if (hB < H) {
+          sm_ml[(warp * H + hB) * 2] = mB;
+          sm_ml[(warp * H + hB) * 2 + 1] = lB;
+        }
+      }
+    }
+  } else if (g < H) {
     float* dst = sm_o + (warp * H + g) * kD + 2 * tq;
 #pragma unroll
     for (int d = 0; d < 16; ++d)
