@@ -85,9 +85,9 @@ METRIC = "index-scan keys/s + sparse decode layer-steps/s; achieved GB/s vs HBM 
 # keyed by (workload, B, kernel). Absent where no capture of the current kernel
 # exists.
 TRAFFIC: dict = {
-    # R=8 capture of fathom_scan_prmt_kernel: 96.56 MB read + 9.77 MB written
+    # R=8 capture of fathom_scan_prmt_kernel: 96.56 MB read + 11.36 MB written
     # per launch (the rest of its scores leave L2 later), x2 for R=16
-    ("qwen3-8b-128k", 92, "fathom_scan_prmt"): 2 * (96_558_080 + 9_770_752),
+    ("qwen3-8b-128k", 92, "fathom_scan_prmt"): 2 * (96_562_432 + 11_357_184),
     # full capture of lightning_scan_kernel<4> at 32 x 80000 tokens x 64 heads
     # (the bench's own workload): 328.70 MB read + 4.64 MB written per launch
     ("minimax-lightning-32x80000", 64, "lightning_scan"): 328_696_832 + 4_638_720,
