@@ -57,22 +57,36 @@ __global__ void __launch_bounds__(256) sparse_gather_kernel(
 }
 
 // The slot of every selected key and the miss count of each (r, g), without
-// moving rows: the attention kernel then reads K/V through these slots.
+// moving rows: the attention kernel then reads K/V through these slots. With
+// vec (k a multiple of 4, idx and slots 16-byte aligned) each thread handles
+// four entries per 16-byte load and store.
 __global__ void __launch_bounds__(256) select_slots_kernel(
     const int32_t* __restrict__ idx, int idx_shared, int G, int k,
     const int32_t* __restrict__ slot_map, int n_max, int32_t* __restrict__ slots,
-    int32_t* __restrict__ misses) {
+    int32_t* __restrict__ misses, int vec) {
+  pdl_wait();
+  pdl_trigger();
   const int u = blockIdx.x;
   const int32_t* irow = idx + (idx_shared ? static_cast<size_t>(u / G) : static_cast<size_t>(u)) * k;
+  const int32_t* smap = slot_map ? slot_map + static_cast<size_t>(u) * n_max : nullptr;
+  int32_t* srow = slots ? slots + static_cast<size_t>(u) * k : nullptr;
+  auto slot_of = [&](int i) { return i < 0 ? -2 : (smap ? smap[i] : -1); };
   int my_misses = 0;
-  for (int j = threadIdx.x; j < k; j += blockDim.x) {
-    const int i = irow[j];
-    int slot = -2;
-    if (i >= 0) {
-      slot = slot_map ? slot_map[static_cast<size_t>(u) * n_max + i] : -1;
-      my_misses += slot < 0 ? 1 : 0;
+  if (vec) {
+    for (int j4 = threadIdx.x; j4 < k / 4; j4 += blockDim.x) {
+      const int4 iv = *reinterpret_cast<const int4*>(irow + 4 * j4);
+      const int4 sv = make_int4(slot_of(iv.x), slot_of(iv.y), slot_of(iv.z), slot_of(iv.w));
+      my_misses += (iv.x >= 0 && sv.x < 0) + (iv.y >= 0 && sv.y < 0) + (iv.z >= 0 && sv.z < 0) +
+                   (iv.w >= 0 && sv.w < 0);
+      if (srow) *reinterpret_cast<int4*>(srow + 4 * j4) = sv;
     }
-    if (slots) slots[static_cast<size_t>(u) * k + j] = slot;
+  } else {
+    for (int j = threadIdx.x; j < k; j += blockDim.x) {
+      const int i = irow[j];
+      const int slot = slot_of(i);
+      my_misses += (i >= 0 && slot < 0) ? 1 : 0;
+      if (srow) srow[j] = slot;
+    }
   }
   __shared__ int warp_sum[8];
   const int w = __reduce_add_sync(0xFFFFFFFFu, my_misses);
@@ -90,7 +104,9 @@ __global__ void __launch_bounds__(256) select_slots_kernel(
 kvs_status select_slots_launch(const int32_t* idx, int idx_shared, int G, int k,
                                const int32_t* slot_map, int n_max, int RG, int32_t* slots,
                                int32_t* misses, cudaStream_t s) {
-  select_slots_kernel<<<RG, 256, 0, s>>>(idx, idx_shared, G, k, slot_map, n_max, slots, misses);
+  const int vec = (k % 4 == 0) && aligned16(idx) && (slots == nullptr || aligned16(slots)) ? 1 : 0;
+  launch_chained(select_slots_kernel, dim3(RG), dim3(256), 0, s, idx, idx_shared, G, k, slot_map, n_max, slots,
+                 misses, vec);
   return check_launch("select_slots");
 }
 
