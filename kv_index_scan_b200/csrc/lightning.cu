@@ -13,23 +13,23 @@
 //  * a producer thread loads 128-token tiles (16 KB) with a 2-D TMA tensor map
 //    over the keys [R * n_max][128 bytes], 128-byte swizzled: each tile lands
 //    in the canonical K-major layout of the MMA's A operand, no conversion;
-//  * the queries of a request become two e4m3 B operands after scaling by a
-//    power of two (exact) that brings max|q| to [2^7, 2^8): hi = e4m3(q 2^e)
-//    and lo = e4m3(q 2^e - hi). A bf16 value has 8 significant bits, so
-//    hi + lo is q 2^e exactly unless lo falls below the e4m3 subnormal range
-//    (elements 2^10 below the largest: an absolute error under 2^-10 there);
+//  * the queries of a request become one e4m3 B operand of 2 Hi rows after
+//    scaling by a power of two (exact) that brings max|q| to [2^7, 2^8):
+//    row h holds hi = e4m3(q_h 2^e) and row Hi + h lo = e4m3(q_h 2^e - hi).
+//    A bf16 value has 8 significant bits, so hi + lo is q 2^e exactly unless
+//    lo falls below the e4m3 subnormal range (elements 2^10 below the
+//    largest: an absolute error under 2^-10 there);
 //  * one elected thread issues tcgen05.mma kind::f8f6f4 (M = 128 tokens,
-//    N = 2 Hi: the hi rows of the query operand, then its lo rows; K = 32 per
-//    instruction, four per tile) into one of up to eight f32 accumulators in
-//    tensor memory; the read-back adds each head's two columns;
+//    N = 2 Hi, K = 32 per instruction, four per tile) into one of up to eight
+//    f32 accumulators in tensor memory;
 //  * sixteen worker warps in four groups of four read the accumulators back,
 //    group g the tiles i = g (mod 4), so that four tiles drain at once: one
 //    token row per thread (warp w reads the TMEM lanes of tokens
-//    32 (w mod 4) .. + 31, every head's two columns), ReLU and the head weights (with
-//    the scale undone), then 32/64/128-token block maxima by warp shuffles and
-//    across the group's warps. The workers also write each request's query
-//    operands up to four tiles ahead of its first tile (two buffers, by
-//    request parity).
+//    32 (w mod 4) .. + 31), each head's hi and lo columns added, ReLU and the
+//    head weights (with the scale undone), then 32/64/128-token block maxima
+//    by warp shuffles and across the group's warps. The workers also write
+//    each request's query operand up to four tiles ahead of its first tile
+//    (two buffers, by request parity).
 // Every wait is bounded; a wait that runs out sets KVS_ETIMEOUT in the status
 // word and the block winds down without leaving copies in flight or TMEM
 // allocated.
