@@ -31,9 +31,11 @@
 //    accumulators by movmatrix.trans (hi parts in the columns of lanes
 //    c < 2, lo parts in those of c >= 2). A head's logit is the sum of its hi
 //    and lo columns; O's two halves are added at the end.
-//  * Online softmax per head inside the four lanes that hold it; the block's
-//    warps merge by log-sum-exp in shared memory, and the blocks (splits) of
-//    one (r, g) in a second small kernel. (Merging the splits inside a
+//  * Online softmax per head: inside the four lanes that hold the head (H > 4),
+//    or across the eight lane groups that hold the tile's tokens, with the
+//    row sums kept per lane until the end (H <= 4). The block's warps merge
+//    by log-sum-exp in shared memory, and the blocks (splits) of one (r, g)
+//    in a second small kernel. (Merging the splits inside a
 //    thread-block cluster instead made the kernel faster alone but the decode
 //    step slower: a clustered launch lost the overlap with its neighbours that
 //    programmatic dependent launch gives the step's kernels.)
