@@ -195,7 +195,7 @@ def test_gather_bit_exact(kvs):
 
 # ----------------------------------------------------------------------------- a5 attention
 
-@pytest.mark.parametrize("H", [1, 4, 8])
+@pytest.mark.parametrize("H", [1, 2, 3, 4, 5, 8])
 @pytest.mark.parametrize("k", [1, 64, 100, 2048])
 @pytest.mark.parametrize("qdt", [torch.float32, torch.bfloat16])
 def test_attention_within_tolerance(kvs, H, k, qdt):

@@ -26,7 +26,7 @@ def kvs():
 
 
 @pytest.mark.parametrize("block", [1, 32, 64, 128])
-@pytest.mark.parametrize("Hi", [64, 16, 128])
+@pytest.mark.parametrize("Hi", [64, 16, 128, 48, 96])
 def test_lightning_scores_within_tolerance(kvs, block, Hi):
     nl = [5000, 1000, 129, 0]
     n_max = 5000
